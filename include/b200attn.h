@@ -1,0 +1,150 @@
+/*
+ * b200attn — causal scaled-dot-product attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libb200attn.so.  Plain pointers and sizes only.
+ *
+ * The operation (both entry points):
+ *   O = softmax(Q K^T * scale + mask) V, per batch b and query head h, where
+ *   query head h reads key/value head h / (H / Hkv) — multi-head (Hkv = H),
+ *   grouped-query (H / Hkv > 1) and multi-query (Hkv = 1) layouts.
+ *   Sources: "Hesper.Layers.Attention" (Mathematical Definition, Multi-Head
+ *   Attention, Causal Masking); "Grouped-Query Attention" §5.1 (one K/V head
+ *   serves group_size query heads, repeat_interleave order) and §5.2 (scores,
+ *   causal bias, softmax, weighted sum); "Causal Multi-Head Self-Attention",
+ *   The causal mask (masked positions get probability exactly zero; every row
+ *   sums to one); "Multi-query attention, annotated" §2.4 and §3 (incremental
+ *   attention against a cache; one shared K/V head).
+ *
+ * Mask: query row i sits at absolute position p_i = start_pos + i (start_pos
+ * = 0 for prefill) and, when causal, sees key j iff j <= p_i; masked keys get
+ * weight exactly 0.  This is the convention of the makarna cached-attention
+ * loop ("attention_cached.go", CausalAttentionCached: new tokens start at
+ * startPos and see every key up to their own position).
+ *
+ * Layouts (all row-major, contiguous, device memory unless stated):
+ *   Q, O : [B, H, Tq, d]
+ *   K, V : [B, Hkv, S_cap, d]   (prefill: S_cap = S = T)
+ *   lse  : [B, H, Tq] float32, optional; lse = max_j s_j + ln sum_j e^{s_j - max}
+ *          over the visible scaled scores s_j (natural log).
+ * Element type: ATTN_F32 (float), ATTN_BF16, ATTN_F16 for Q, K, V and O alike;
+ * accumulation is always float32.  Output is rounded to nearest-even.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates nothing on
+ * the device, never synchronises inside a call, and enqueues its kernels on
+ * `stream` (a cudaStream_t; NULL = legacy default stream).  It keeps no state
+ * between calls except read-only kernel attributes.
+ *
+ * Errors: every argument is checked before anything is enqueued; on any error
+ * nothing is launched and O is left untouched.  Nothing aborts the process.
+ *   ATTN_ERR_INVALID_ARG  null pointer with a non-empty problem, negative size,
+ *                         Hkv = 0, H % Hkv != 0, S > S_cap, start_pos < 0,
+ *                         start_pos + Tnew > S, non-finite scale, a pointer not
+ *                         aligned to 16 bytes, or d <= 0;
+ *   ATTN_ERR_UNSUPPORTED  d > 256;
+ *   ATTN_ERR_WORKSPACE    workspace smaller than attn_cached_workspace_size();
+ *   ATTN_ERR_CUDA         a CUDA runtime error while encoding or launching;
+ *   ATTN_ERR_DEVICE_TIMEOUT reported by attn_device_status() when a kernel gave
+ *                         up a bounded wait (it then exits cleanly).
+ * A problem with B * H * Tq = 0 returns ATTN_OK and launches nothing.
+ */
+#ifndef B200ATTN_H
+#define B200ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,
+    ATTN_ERR_UNSUPPORTED = 2,
+    ATTN_ERR_WORKSPACE = 3,
+    ATTN_ERR_CUDA = 4,
+    ATTN_ERR_DEVICE_TIMEOUT = 5
+} attn_status_t;
+
+typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1, ATTN_F16 = 2 } attn_dtype_t;
+
+/* Which kernel family a call uses (see attn_prefill_plan / attn_cached_plan). */
+typedef enum {
+    ATTN_KERNEL_NONE = 0,        /* empty problem: nothing launched            */
+    ATTN_KERNEL_SIMT = 1,        /* float32 CUDA-core kernel (any d <= 256)    */
+    ATTN_KERNEL_TCGEN05 = 2,     /* TMA + tcgen05/TMEM fused prefill kernel    */
+    ATTN_KERNEL_SPLITKV = 3      /* split-KV decode kernel + LSE combine       */
+} attn_kernel_t;
+
+/*
+ * Full-sequence attention ("Hesper.Layers.Attention", forward, steps 4-6;
+ * "Causal Multi-Head Self-Attention", Dataflow and shapes).
+ *   q [B,H,T,d], k/v [B,Hkv,T,d], o [B,H,T,d]; lse nullable [B,H,T].
+ *   causal != 0: row i sees keys 0..i; causal = 0: every key.
+ * Equivalent to attn_cached with Tnew = S = S_cap = T and start_pos = 0.
+ */
+ATTN_API attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                           attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t T,
+                           int64_t d, float scale, int causal, void* stream);
+
+/*
+ * KV-cached attention ("Multi-query attention, annotated" §2.4: new queries
+ * against the cached keys and values; "attention_cached.go",
+ * CausalAttentionCached).  The history already holds the new tokens' keys and
+ * values at positions start_pos .. start_pos + Tnew - 1.
+ *   q [B,H,Tnew,d]; k_hist/v_hist [B,Hkv,S_cap,d], first S rows valid;
+ *   o [B,H,Tnew,d]; lse nullable [B,H,Tnew].  Always causal.
+ *   workspace: device buffer of at least attn_cached_workspace_size() bytes,
+ *   16-byte aligned (may be NULL when that size is 0); its contents on entry
+ *   do not matter and are clobbered.
+ */
+ATTN_API attn_status_t attn_cached(const void* q, const void* k_hist, const void* v_hist, void* o,
+                          float* lse, attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                          int64_t Tnew, int64_t S, int64_t S_cap, int64_t d, int64_t start_pos,
+                          float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace attn_cached needs for this problem (0 if none).  Pure
+ * host arithmetic; valid without a GPU.  Returns 0 for arguments that
+ * attn_cached would reject. */
+ATTN_API size_t attn_cached_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                                  int64_t Tnew, int64_t S, int64_t d, int64_t start_pos);
+
+/* Kernel family the call with these arguments would use; host-only, no GPU
+ * needed.  Returns ATTN_KERNEL_NONE for an empty problem and -1 cast to
+ * attn_kernel_t for arguments the entry point would reject. */
+ATTN_API attn_kernel_t attn_prefill_plan(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t T,
+                                int64_t d, int causal);
+ATTN_API attn_kernel_t attn_cached_plan(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                               int64_t Tnew, int64_t S, int64_t S_cap, int64_t d,
+                               int64_t start_pos);
+
+/* Human-readable name of a status code (static string, never NULL). */
+ATTN_API const char* attn_status_string(attn_status_t status);
+
+/*
+ * Device-side status.  Every wait inside the kernels is bounded; a wait that
+ * runs out records ATTN_ERR_DEVICE_TIMEOUT in a per-device status word and
+ * the kernel exits cleanly, leaving the context usable.  This call
+ * synchronises `stream`, returns the recorded status (ATTN_OK if none) and,
+ * if `reset` != 0, clears it.  Unlike the compute calls it blocks the host.
+ */
+ATTN_API attn_status_t attn_device_status(void* stream, int reset);
+
+/* Bound for every device-side wait, in nanoseconds (default 2e9).  Tests
+ * shorten it; 0 restores the default.  Host-side setting read at launch. */
+ATTN_API void attn_set_wait_timeout_ns(uint64_t ns);
+
+/* Library version, as major * 10000 + minor * 100 + patch. */
+ATTN_API int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* B200ATTN_H */

@@ -1,0 +1,149 @@
+"""The C-ABI library without a GPU: it loads, exports every function the
+header declares, and rejects bad arguments before touching the device.
+
+Only host-side code paths are exercised here (argument checks, planning,
+workspace sizing, status strings); no call in this file launches a kernel.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from transformer_attention_causal_b200 import _lib
+    from transformer_attention_causal_b200.build import build
+
+    build()
+    return _lib.load()
+
+
+def declared_functions():
+    names = []
+    for fname in os.listdir(HEADER_DIR):
+        if fname.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, fname)).read()
+            names += re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for required in ("attn_prefill", "attn_cached", "attn_cached_workspace_size",
+                     "attn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from transformer_attention_causal_b200 import _lib
+
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(declared_functions()) <= exported
+    # nothing but the ABI is exported from the library's own code
+    assert {n for n in exported if n.startswith("attn_")} == set(declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    from transformer_attention_causal_b200 import _lib
+
+    for code in range(6):
+        assert isinstance(_lib.status_string(code), str) and _lib.status_string(code)
+    assert _lib.status_string(99) == "unknown status"
+    assert lib.attn_version() >= 100
+
+
+F32, BF16, F16 = 0, 1, 2
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def prefill(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, dt=BF16, B=1, H=4, Hkv=2, T=8, d=64,
+            scale=0.125, causal=1):
+    return lib.attn_prefill(q, k, v, o, lse, dt, B, H, Hkv, T, d, scale, causal, None)
+
+
+def cached(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, dt=BF16, B=1, H=4, Hkv=2, Tnew=1, S=8,
+           S_cap=8, d=64, start_pos=7, scale=0.125, ws=None, ws_bytes=0):
+    return lib.attn_cached(q, k, v, o, lse, dt, B, H, Hkv, Tnew, S, S_cap, d, start_pos, scale, ws,
+                           ws_bytes, None)
+
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+
+
+@pytest.mark.parametrize("kwargs", [
+    dict(q=None), dict(k=None), dict(v=None), dict(o=None),
+    dict(q=MISALIGNED), dict(o=MISALIGNED), dict(lse=ctypes.c_void_p(0x10002)),
+    dict(B=-1), dict(H=-2), dict(T=-1), dict(d=-8), dict(d=0),
+    dict(Hkv=0), dict(H=6, Hkv=4), dict(dt=7),
+    dict(scale=float("nan")), dict(scale=float("inf")),
+])
+def test_prefill_rejects_invalid_arguments(lib, kwargs):
+    assert prefill(lib, **kwargs) == INVALID
+
+
+def test_prefill_rejects_oversized_head(lib):
+    assert prefill(lib, d=264) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("kwargs", [
+    dict(start_pos=8),                 # start_pos + Tnew > S
+    dict(S=9, S_cap=8, start_pos=8),   # S > S_cap
+    dict(start_pos=-1),
+    dict(Tnew=3, start_pos=6),         # 6 + 3 > 8
+    dict(q=None), dict(k=MISALIGNED),
+])
+def test_cached_rejects_invalid_arguments(lib, kwargs):
+    assert cached(lib, **kwargs) == INVALID
+
+
+def test_cached_reports_a_short_workspace(lib):
+    need = lib.attn_cached_workspace_size(BF16, 64, 32, 8, 1, 8192, 128, 8191)
+    assert need > 0
+    args = dict(B=64, H=32, Hkv=8, Tnew=1, S=8192, S_cap=8192, d=128, start_pos=8191)
+    assert cached(lib, ws=None, ws_bytes=0, **args) == WORKSPACE
+    assert cached(lib, ws=FAKE, ws_bytes=need - 1, **args) == WORKSPACE
+    assert cached(lib, ws=MISALIGNED, ws_bytes=need, **args) == INVALID
+
+
+def test_empty_problems_are_a_no_op(lib):
+    # B * H * Tq == 0: nothing is launched, null pointers allowed
+    assert prefill(lib, q=None, k=None, v=None, o=None, B=0) == 0
+    assert prefill(lib, q=None, k=None, v=None, o=None, T=0) == 0
+    assert cached(lib, q=None, k=None, v=None, o=None, Tnew=0, start_pos=8) == 0
+    assert lib.attn_prefill_plan(BF16, 0, 4, 2, 8, 64, 1) == 0
+
+
+def test_plans_pick_the_intended_kernels(lib):
+    from transformer_attention_causal_b200 import _lib as L
+
+    # float32 always runs on CUDA cores
+    assert lib.attn_prefill_plan(F32, 1, 2, 1, 16, 8, 1) == L.KERNEL_SIMT
+    # the four 16-bit workloads
+    assert lib.attn_prefill_plan(BF16, 1, 32, 32, 2048, 80, 1) == L.KERNEL_TCGEN05
+    assert lib.attn_prefill_plan(BF16, 8, 16, 8, 4096, 128, 1) == L.KERNEL_TCGEN05
+    assert lib.attn_cached_plan(BF16, 64, 32, 8, 1, 8192, 8192, 128, 8191) == L.KERNEL_SPLITKV
+    assert lib.attn_cached_plan(F16, 32, 8, 1, 512, 4096, 4096, 128, 3584) == L.KERNEL_TCGEN05
+    # head sizes the tensor-core kernel does not take fall back to CUDA cores
+    assert lib.attn_prefill_plan(BF16, 1, 2, 1, 16, 40, 1) == L.KERNEL_SIMT
+    assert lib.attn_prefill_plan(BF16, 1, 2, 1, 16, 200, 1) == L.KERNEL_SIMT
+    # rejected arguments
+    assert lib.attn_prefill_plan(BF16, 1, 3, 2, 16, 64, 1) == -1
+
+
+def test_workspace_size_is_zero_without_splits(lib):
+    # a single long sequence on one K/V head still splits; a tiny history does not
+    assert lib.attn_cached_workspace_size(BF16, 1, 4, 4, 1, 64, 128, 63) == 0
+    assert lib.attn_cached_workspace_size(BF16, 1, 4, 1, 1, 65536, 128, 65535) > 0
+    # rejected arguments report 0
+    assert lib.attn_cached_workspace_size(BF16, 1, 4, 3, 1, 64, 128, 63) == 0

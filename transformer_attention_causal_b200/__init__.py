@@ -1,5 +1,134 @@
 """B200-native causal (MHA / GQA / MQA) scaled-dot-product attention.
 
-The compute lives in ``libb200attn.so`` (CUDA C++ for sm_100a behind a C ABI,
-declared in ``include/b200attn.h``); this package is a thin binding to it.
+The compute lives in ``libb200attn.so`` (CUDA C++ for sm_100a behind the C ABI
+declared in ``include/b200attn.h``).  This package only marshals arguments:
+torch supplies device memory and the current stream; every step of the
+attention runs in the library's kernels.
+
+    prefill(q, k, v, scale=..., causal=True)        q [B,H,T,d], k/v [B,Hkv,T,d]
+    cached(q, k_hist, v_hist, start_pos=..., scale=...)
+                                                    q [B,H,Tnew,d], k/v [B,Hkv,S_cap,d]
 """
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import AttnError
+
+__all__ = ["prefill", "cached", "cached_workspace_size", "prefill_plan", "cached_plan",
+           "device_status", "set_wait_timeout_ns", "AttnError"]
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return _lib.F32
+    if t.dtype == torch.bfloat16:
+        return _lib.BF16
+    if t.dtype == torch.float16:
+        return _lib.F16
+    raise TypeError(f"unsupported dtype {t.dtype}: expected float32, bfloat16 or float16")
+
+
+def _code_of(dtype) -> int:
+    torch = _torch()
+    return {torch.float32: _lib.F32, torch.bfloat16: _lib.BF16, torch.float16: _lib.F16}[dtype]
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(*tensors):
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def prefill(q, k, v, *, scale: float, causal: bool = True, out=None, lse=None, stream=None):
+    """Full-sequence attention.  q [B,H,T,d]; k, v [B,Hkv,T,d]; returns O [B,H,T,d].
+    ``lse`` (optional float32 [B,H,T]) receives the log-sum-exp of each row."""
+    _check(q, k, v, out, lse)
+    B, H, T, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (B, Hkv, T, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, Hkv, T, d] matching q")
+    if out is None:
+        out = q.new_empty(q.shape)
+    st = _lib.load().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _dtype_code(q),
+                                  B, H, Hkv, T, d, float(scale), int(bool(causal)),
+                                  _stream_handle(stream, q.device))
+    if st != _lib.OK:
+        raise AttnError(st, "attn_prefill")
+    return out
+
+
+def cached_workspace_size(dtype, B, H, Hkv, Tnew, S, d, start_pos) -> int:
+    return int(_lib.load().attn_cached_workspace_size(_code_of(dtype), B, H, Hkv, Tnew, S, d,
+                                                       start_pos))
+
+
+def cached(q, k_hist, v_hist, *, start_pos: int, scale: float, S: int | None = None, out=None,
+           lse=None, workspace=None, stream=None):
+    """New tokens at ``start_pos`` against a K/V history that already holds them.
+    q [B,H,Tnew,d]; k_hist, v_hist [B,Hkv,S_cap,d] (first S rows valid, default
+    S = S_cap).  ``workspace`` (uint8 CUDA tensor) is allocated here when not given."""
+    _check(q, k_hist, v_hist, out, lse, workspace)
+    B, H, Tnew, d = q.shape
+    Hkv, S_cap = k_hist.shape[1], k_hist.shape[2]
+    if tuple(v_hist.shape) != tuple(k_hist.shape) or k_hist.shape[0] != B or k_hist.shape[3] != d:
+        raise ValueError("k_hist and v_hist must be [B, Hkv, S_cap, d] matching q")
+    S = S_cap if S is None else int(S)
+    if out is None:
+        out = q.new_empty(q.shape)
+    need = cached_workspace_size(q.dtype, B, H, Hkv, Tnew, S, d, start_pos)
+    if workspace is None and need > 0:
+        workspace = _torch().empty(need, dtype=_torch().uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.load().attn_cached(_ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(out), _ptr(lse),
+                                 _dtype_code(q), B, H, Hkv, Tnew, S, S_cap, d, int(start_pos),
+                                 float(scale), _ptr(workspace), ws_bytes,
+                                 _stream_handle(stream, q.device))
+    if st != _lib.OK:
+        raise AttnError(st, "attn_cached")
+    return out
+
+
+def prefill_plan(dtype, B, H, Hkv, T, d, causal=True) -> str:
+    k = _lib.load().attn_prefill_plan(_code_of(dtype), B, H, Hkv, T, d, int(bool(causal)))
+    return _lib.KERNEL_NAMES[k]
+
+
+def cached_plan(dtype, B, H, Hkv, Tnew, S, S_cap, d, start_pos) -> str:
+    k = _lib.load().attn_cached_plan(_code_of(dtype), B, H, Hkv, Tnew, S, S_cap, d, start_pos)
+    return _lib.KERNEL_NAMES[k]
+
+
+def device_status(stream=None, reset: bool = True) -> int:
+    """Synchronise the stream and return (and by default clear) the device
+    status word: 0 = OK, 5 = a bounded device-side wait ran out."""
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(_lib.load().attn_device_status(ctypes.c_void_p(s.cuda_stream), int(bool(reset))))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _lib.load().attn_set_wait_timeout_ns(int(ns))

@@ -1,0 +1,442 @@
+// libb200attn: C-ABI entry points, argument checks, planning and launches.
+// The operation, layouts, ownership and error rules are documented in
+// include/b200attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+#include <type_traits>
+
+#include "b200attn.h"
+#include "decode_splitkv.cuh"
+#include "prefill_tcgen05.cuh"
+#include "simt_attn.cuh"
+
+using namespace b200attn;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+
+// Planning constants for B200: 148 SMs, two decode CTAs resident per SM.
+constexpr int kPlanSMs = 148;
+constexpr int kDecodeCtasPerSM = 2;
+constexpr int kDecodeStageKeys = 64;
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
+size_t esize(attn_dtype_t dt) { return dt == ATTN_F32 ? 4 : 2; }
+
+struct Problem {
+    attn_dtype_t dt;
+    int64_t B, H, Hkv, Tq, S, S_cap, d, start_pos;
+    int causal;
+    bool cached;  // attn_cached: split-KV decode allowed
+};
+
+struct Plan {
+    attn_kernel_t kernel = ATTN_KERNEL_NONE;
+    // split-KV decode
+    int R = 0, Rv = 0, nsplit = 1;
+    int64_t chunk = 0, kv_end = 0;
+    size_t ws_bytes = 0;
+    // tcgen05 prefill
+    int dch = 0, pair_mode = 0, n_qb = 0, units_per_level = 0, n_levels = 0;
+};
+
+bool empty_problem(const Problem& pb) { return pb.B == 0 || pb.H == 0 || pb.Tq == 0; }
+
+// Shape checks shared by every entry point (pointers are checked separately).
+attn_status_t check_shape(const Problem& pb) {
+    if (pb.dt != ATTN_F32 && pb.dt != ATTN_BF16 && pb.dt != ATTN_F16) return ATTN_ERR_INVALID_ARG;
+    if (pb.B < 0 || pb.H < 0 || pb.Hkv < 0 || pb.Tq < 0 || pb.S < 0 || pb.S_cap < 0 ||
+        pb.d < 0 || pb.start_pos < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (empty_problem(pb)) return ATTN_OK;
+    if (pb.Hkv == 0 || pb.H % pb.Hkv != 0 || pb.d == 0) return ATTN_ERR_INVALID_ARG;
+    if (pb.S > pb.S_cap || pb.start_pos + pb.Tq > pb.S) return ATTN_ERR_INVALID_ARG;
+    if (pb.d > kSimtMaxD) return ATTN_ERR_UNSUPPORTED;
+    // 32-bit grid and index limits of the kernels
+    if (pb.B * pb.H * pb.Tq > (int64_t(1) << 40) || pb.B * pb.Hkv > (int64_t(1) << 30))
+        return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+int decode_rmax(int64_t d) {
+    if (d == 64 || d == 128) return 16;
+    if (d == 256) return 8;
+    return 0;
+}
+
+int next_pow2_at_least4(int64_t x) {
+    int r = 4;
+    while (r < x) r <<= 1;
+    return r;
+}
+
+void plan_decode(const Problem& pb, Plan& pl) {
+    pl.kernel = ATTN_KERNEL_SPLITKV;
+    const int64_t G = pb.H / pb.Hkv;
+    pl.Rv = int(G * pb.Tq);
+    pl.R = next_pow2_at_least4(pl.Rv);
+    pl.kv_end = std::min<int64_t>(pb.S, pb.start_pos + pb.Tq);
+    const int64_t tiles = (pl.kv_end + kDecodeStageKeys - 1) / kDecodeStageKeys;
+    const int64_t units = pb.B * pb.Hkv;
+    const int64_t slots = int64_t(kPlanSMs) * kDecodeCtasPerSM;
+    // Pick the split count that fills the last wave of CTAs best; prefer fewer
+    // splits on ties and keep at least 4 stages per split when there is room.
+    int best_n = 1;
+    double best_score = -1.0;
+    const int64_t max_n = std::max<int64_t>(1, std::min<int64_t>(tiles, 128));
+    for (int64_t n = 1; n <= max_n; ++n) {
+        const int64_t per = (tiles + n - 1) / n;
+        const int64_t n_eff = (tiles + per - 1) / per;  // no empty splits
+        if (n_eff != n) continue;
+        if (per < 4 && n > 1 && units * (n - 1) >= slots) continue;
+        const int64_t ctas = units * n;
+        const int64_t waves = (ctas + slots - 1) / slots;
+        const double fill = double(ctas) / double(waves * slots);
+        const double score = fill - 0.002 * double(n);
+        if (score > best_score + 1e-12) {
+            best_score = score;
+            best_n = int(n);
+        }
+    }
+    const int64_t per = (tiles + best_n - 1) / best_n;
+    pl.nsplit = best_n;
+    pl.chunk = per * kDecodeStageKeys;
+    pl.ws_bytes = 0;
+    if (pl.nsplit > 1) {
+        const size_t rows = size_t(units) * pl.nsplit * pl.Rv;
+        const size_t bytes = rows * size_t(pb.d + 2) * sizeof(float);
+        pl.ws_bytes = (bytes + 255) & ~size_t(255);
+    }
+}
+
+void plan_prefill_tc(const Problem& pb, Plan& pl) {
+    pl.kernel = ATTN_KERNEL_TCGEN05;
+    const int64_t G = pb.H / pb.Hkv;
+    pl.dch = pb.d <= 64 ? 1 : 2;
+    pl.pair_mode = (G % 2 == 0) ? 0 : 1;
+    pl.n_qb = int((pb.Tq + 127) / 128);
+    if (pl.pair_mode == 0) {
+        pl.units_per_level = int(pb.B * pb.Hkv * (G / 2));
+        pl.n_levels = pl.n_qb;
+    } else {
+        pl.units_per_level = int(pb.B * pb.H);
+        pl.n_levels = (pl.n_qb + 1) / 2;
+    }
+}
+
+attn_status_t make_plan(const Problem& pb, Plan& pl) {
+    attn_status_t st = check_shape(pb);
+    if (st != ATTN_OK) return st;
+    pl = Plan();
+    if (empty_problem(pb)) return ATTN_OK;
+    if (pb.dt == ATTN_F32) {
+        pl.kernel = ATTN_KERNEL_SIMT;
+        return ATTN_OK;
+    }
+    const int64_t G = pb.H / pb.Hkv;
+    const int rmax = decode_rmax(pb.d);
+    if (pb.cached && rmax > 0 && G * pb.Tq <= rmax) {
+        plan_decode(pb, pl);
+        return ATTN_OK;
+    }
+    if (pb.d % 16 == 0 && pb.d >= 64 && pb.d <= 128 &&
+        (pb.B * pb.Hkv * std::max<int64_t>(G / 2, 1) * ((pb.Tq + 127) / 128)) < (int64_t(1) << 31) &&
+        pb.S_cap * pb.d * 2 < (int64_t(1) << 40)) {
+        plan_prefill_tc(pb, pl);
+        return ATTN_OK;
+    }
+    pl.kernel = ATTN_KERNEL_SIMT;
+    return ATTN_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+attn_status_t get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// [nslices, rows (pitch row_pitch), d] 16-bit tensor, box of 64 columns x 128 rows.
+attn_status_t encode_rows(CUtensorMap* map, const void* ptr, attn_dtype_t dt, int64_t d,
+                          int64_t rows, int64_t row_pitch, int64_t nslices) {
+    const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(nslices)};
+    const cuuint64_t strides[2] = {cuuint64_t(d * 2), cuuint64_t(row_pitch * d * 2)};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapDataType ty =
+        dt == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = g_encode(map, ty, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ launches
+
+template <typename K>
+attn_status_t set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) ==
+                   cudaSuccess
+               ? ATTN_OK
+               : ATTN_ERR_CUDA;
+}
+
+attn_status_t launch_status() {
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename T>
+attn_status_t run_simt(const Problem& pb, const void* q, const void* k, const void* v, void* o,
+                       float* lse, float scale, cudaStream_t stream) {
+    SimtParams sp;
+    sp.q = q; sp.k = k; sp.v = v; sp.o = o; sp.lse = lse;
+    sp.B = pb.B; sp.H = pb.H; sp.Hkv = pb.Hkv; sp.Tq = pb.Tq; sp.S = pb.S; sp.S_cap = pb.S_cap;
+    sp.d = pb.d; sp.start_pos = pb.start_pos; sp.scale = scale; sp.causal = pb.causal;
+    const int64_t rows = pb.B * pb.H * pb.Tq;
+    const int64_t blocks = (rows + kSimtWarps - 1) / kSimtWarps;
+    if (blocks > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+    simt_attention_kernel<T><<<unsigned(blocks), kSimtWarps * 32, 0, stream>>>(sp);
+    return launch_status();
+}
+
+template <typename T, int D, int R>
+attn_status_t launch_decode_R(const DecodeParams& dp, cudaStream_t stream) {
+    constexpr size_t smem = DecodeShape<D, R>::smem_bytes(sizeof(T));
+    auto kern = decode_splitkv_kernel<T, D, R>;
+    static std::once_flag once[8];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    attn_status_t st = ATTN_OK;
+    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
+    if (st != ATTN_OK) return st;
+    dim3 grid(unsigned(dp.nsplit), unsigned(dp.B * dp.Hkv));
+    kern<<<grid, 160, smem, stream>>>(dp);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
+    if (dp.nsplit > 1) {
+        const int64_t rows = int64_t(dp.B) * dp.Hkv * dp.Rv;
+        decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, stream>>>(dp);
+        return launch_status();
+    }
+    return ATTN_OK;
+}
+
+template <typename T, int D>
+attn_status_t launch_decode_D(int R, const DecodeParams& dp, cudaStream_t stream) {
+    switch (R) {
+    case 4: return launch_decode_R<T, D, 4>(dp, stream);
+    case 8: return launch_decode_R<T, D, 8>(dp, stream);
+    case 16:
+        if constexpr (D <= 128) return launch_decode_R<T, D, 16>(dp, stream);
+        return ATTN_ERR_UNSUPPORTED;
+    default: return ATTN_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const void* k,
+                         const void* v, void* o, float* lse, float scale, void* ws,
+                         cudaStream_t stream) {
+    DecodeParams dp;
+    dp.q = q; dp.k = k; dp.v = v; dp.o = o; dp.lse = lse;
+    const size_t rows = size_t(pb.B * pb.Hkv) * pl.nsplit * pl.Rv;
+    float* wsf = static_cast<float*>(ws);
+    dp.ws_o = wsf;
+    dp.ws_m = wsf ? wsf + rows * pb.d : nullptr;
+    dp.ws_l = wsf ? dp.ws_m + rows : nullptr;
+    dp.B = int(pb.B); dp.H = int(pb.H); dp.Hkv = int(pb.Hkv);
+    dp.G = int(pb.H / pb.Hkv); dp.Tnew = int(pb.Tq); dp.Rv = pl.Rv;
+    dp.S = pb.S; dp.S_cap = pb.S_cap; dp.start_pos = pb.start_pos;
+    dp.kv_end = pl.kv_end; dp.chunk = pl.chunk; dp.nsplit = pl.nsplit;
+    dp.scale_log2 = scale * 1.4426950408889634f;
+    dp.timeout_ns = g_timeout_ns.load();
+    switch (pb.d) {
+    case 64: return launch_decode_D<T, 64>(pl.R, dp, stream);
+    case 128: return launch_decode_D<T, 128>(pl.R, dp, stream);
+    case 256: return launch_decode_D<T, 256>(pl.R, dp, stream);
+    default: return ATTN_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T, int DCH>
+attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q, const void* k,
+                                const void* v, void* o, float* lse, float scale,
+                                cudaStream_t stream) {
+    if (get_encoder() != ATTN_OK) return ATTN_ERR_CUDA;
+    CUtensorMap mq, mk, mv;
+    if (encode_rows(&mq, q, pb.dt, pb.d, pb.Tq, pb.Tq, pb.B * pb.H) != ATTN_OK ||
+        encode_rows(&mk, k, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK ||
+        encode_rows(&mv, v, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK)
+        return ATTN_ERR_CUDA;
+    PrefillParams pp;
+    pp.o = o; pp.lse = lse;
+    pp.B = int(pb.B); pp.H = int(pb.H); pp.Hkv = int(pb.Hkv); pp.G = int(pb.H / pb.Hkv);
+    pp.Tq = int(pb.Tq); pp.S = pb.S; pp.start_pos = pb.start_pos; pp.d = int(pb.d);
+    pp.causal = pb.causal; pp.pair_mode = pl.pair_mode; pp.n_qb = pl.n_qb;
+    pp.units_per_level = pl.units_per_level;
+    pp.scale_log2 = scale * 1.4426950408889634f;
+    pp.timeout_ns = g_timeout_ns.load();
+    constexpr size_t smem = prefill_smem_bytes<DCH>();
+    auto kern = prefill_tcgen05_kernel<T, DCH>;
+    static std::once_flag once[8];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    attn_status_t st = ATTN_OK;
+    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
+    if (st != ATTN_OK) return st;
+    const int64_t grid = int64_t(pl.units_per_level) * pl.n_levels;
+    kern<<<unsigned(grid), kPfThreads, smem, stream>>>(mq, mk, mv, pp);
+    return launch_status();
+}
+
+template <typename T>
+attn_status_t run_prefill_tc(const Problem& pb, const Plan& pl, const void* q, const void* k,
+                             const void* v, void* o, float* lse, float scale,
+                             cudaStream_t stream) {
+    if (pl.dch == 1) return launch_prefill_tc<T, 1>(pb, pl, q, k, v, o, lse, scale, stream);
+    return launch_prefill_tc<T, 2>(pb, pl, q, k, v, o, lse, scale, stream);
+}
+
+attn_status_t dispatch(const Problem& pb, const Plan& pl, const void* q, const void* k,
+                       const void* v, void* o, float* lse, float scale, void* ws,
+                       cudaStream_t stream) {
+    switch (pl.kernel) {
+    case ATTN_KERNEL_NONE: return ATTN_OK;
+    case ATTN_KERNEL_SIMT:
+        if (pb.dt == ATTN_F32) return run_simt<float>(pb, q, k, v, o, lse, scale, stream);
+        if (pb.dt == ATTN_BF16) return run_simt<__nv_bfloat16>(pb, q, k, v, o, lse, scale, stream);
+        return run_simt<__half>(pb, q, k, v, o, lse, scale, stream);
+    case ATTN_KERNEL_SPLITKV:
+        if (pb.dt == ATTN_BF16)
+            return run_decode<__nv_bfloat16>(pb, pl, q, k, v, o, lse, scale, ws, stream);
+        return run_decode<__half>(pb, pl, q, k, v, o, lse, scale, ws, stream);
+    case ATTN_KERNEL_TCGEN05:
+        if (pb.dt == ATTN_BF16)
+            return run_prefill_tc<__nv_bfloat16>(pb, pl, q, k, v, o, lse, scale, stream);
+        return run_prefill_tc<__half>(pb, pl, q, k, v, o, lse, scale, stream);
+    }
+    return ATTN_ERR_INVALID_ARG;
+}
+
+attn_status_t check_pointers(const Problem& pb, const void* q, const void* k, const void* v,
+                             const void* o, const float* lse) {
+    if (empty_problem(pb)) return ATTN_OK;
+    if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (lse && !aligned4(lse)) return ATTN_ERR_INVALID_ARG;
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                           attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t T,
+                           int64_t d, float scale, int causal, void* stream) {
+    Problem pb{dtype, B, H, Hkv, T, T, T, d, 0, causal ? 1 : 0, false};
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    Plan pl;
+    attn_status_t st = make_plan(pb, pl);
+    if (st != ATTN_OK) return st;
+    st = check_pointers(pb, q, k, v, o, lse);
+    if (st != ATTN_OK) return st;
+    return dispatch(pb, pl, q, k, v, o, lse, scale, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_cached(const void* q, const void* k_hist, const void* v_hist, void* o,
+                          float* lse, attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                          int64_t Tnew, int64_t S, int64_t S_cap, int64_t d, int64_t start_pos,
+                          float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    Problem pb{dtype, B, H, Hkv, Tnew, S, S_cap, d, start_pos, 1, true};
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    Plan pl;
+    attn_status_t st = make_plan(pb, pl);
+    if (st != ATTN_OK) return st;
+    st = check_pointers(pb, q, k_hist, v_hist, o, lse);
+    if (st != ATTN_OK) return st;
+    if (pl.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < pl.ws_bytes) return ATTN_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+    }
+    return dispatch(pb, pl, q, k_hist, v_hist, o, lse, scale, workspace,
+                    static_cast<cudaStream_t>(stream));
+}
+
+size_t attn_cached_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                                  int64_t Tnew, int64_t S, int64_t d, int64_t start_pos) {
+    Problem pb{dtype, B, H, Hkv, Tnew, S, S, d, start_pos, 1, true};
+    Plan pl;
+    if (make_plan(pb, pl) != ATTN_OK) return 0;
+    return pl.ws_bytes;
+}
+
+attn_kernel_t attn_prefill_plan(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t T,
+                                int64_t d, int causal) {
+    Problem pb{dtype, B, H, Hkv, T, T, T, d, 0, causal ? 1 : 0, false};
+    Plan pl;
+    if (make_plan(pb, pl) != ATTN_OK) return static_cast<attn_kernel_t>(-1);
+    return pl.kernel;
+}
+
+attn_kernel_t attn_cached_plan(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                               int64_t Tnew, int64_t S, int64_t S_cap, int64_t d,
+                               int64_t start_pos) {
+    Problem pb{dtype, B, H, Hkv, Tnew, S, S_cap, d, start_pos, 1, true};
+    Plan pl;
+    if (make_plan(pb, pl) != ATTN_OK) return static_cast<attn_kernel_t>(-1);
+    return pl.kernel;
+}
+
+const char* attn_status_string(attn_status_t status) {
+    switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape";
+    case ATTN_ERR_WORKSPACE: return "workspace too small";
+    case ATTN_ERR_CUDA: return "CUDA runtime error";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "a device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+attn_status_t attn_device_status(void* stream, int reset) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int value = 0;
+    if (cudaMemcpyFromSymbolAsync(&value, g_device_status, sizeof(value), 0,
+                                  cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (reset && value != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0,
+                                    cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+    }
+    return static_cast<attn_status_t>(value);
+}
+
+void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs); }
+
+int attn_version(void) { return 100; }
+
+}  // extern "C"

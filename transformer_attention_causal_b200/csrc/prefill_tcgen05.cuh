@@ -1,0 +1,389 @@
+// Fused causal prefill attention on the 5th-generation tensor cores.
+//
+// Q.K^T and P.V are real dense contractions, so both run as tcgen05 MMAs
+// with fp32 accumulators in tensor memory (TMEM); the softmax between them is
+// the online form ("Causal Multi-Head Self-Attention", Two exact
+// full-sequence algorithms: running row maximum and exponential sum, updated
+// as each key tile arrives) with exp2 and the scale folded into the exponent.
+//
+// CTA work unit = two "slots", each a 128-query-row tile of one head:
+//   * group size G even: two query heads of the same K/V head, same rows, so
+//     every K/V tile loaded to shared memory feeds both heads ("Grouped-Query
+//     Attention" §5.1 without the repeat_interleave copy);
+//   * G odd (MHA, G = 1): one head, two consecutive 128-row tiles.
+// Units are launched heaviest first (longest causal row range first).
+//
+// Warp roles (12 warps):
+//   warp 0      TMA producer: Q tiles once, then K_n, V_n into a ring of NST
+//               128-key stages (128-byte swizzle, zero fill past the end);
+//   warp 1      TMEM owner (allocates all 512 columns) and single-thread MMA
+//               issuer: S_s = Q_s K_n^T (SS MMA, M=N=128), O_s += P_s V_n
+//               (TS MMA: P read straight from TMEM, N = d);
+//   warps 4-7   softmax for slot 0, warps 8-11 softmax for slot 1: one
+//               thread per query row (TMEM lane), 128 scores in registers.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512);
+// P_s (16-bit, two per column) overwrites the first 64 columns of S_s.
+// Order per key tile n (two slots ping-pong so one slot's softmax overlaps
+// the other slot's MMAs):  wait P_0(n) -> O_0 += P_0 V_n -> S_0(n+1);
+//                          wait P_1(n) -> O_1 += P_1 V_n -> S_1(n+1).
+// Key tiles entirely above the diagonal are never loaded; only tiles that
+// straddle the diagonal (or the end of the keys) are masked.
+//
+// The running maximum is updated lazily: it is only raised (and O rescaled in
+// TMEM) when the tile maximum exceeds it by more than 2^8 in the exp2 domain;
+// otherwise the stale maximum keeps every P below 256, exact after the final
+// division by l.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace b200attn {
+
+struct PrefillParams {
+    void* o;
+    float* lse;
+    int B, H, Hkv, G, Tq;
+    int64_t S;           // keys 0..S-1 exist
+    int64_t start_pos;   // absolute position of query row 0
+    int d;
+    int causal;
+    int pair_mode;       // 0: two heads share a row tile; 1: one head, two row tiles
+    int n_qb;            // ceil(Tq / 128)
+    int units_per_level;
+    float scale_log2;    // scale * log2(e)
+    uint64_t timeout_ns;
+};
+
+constexpr int kPfThreads = 384;
+constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 16-bit columns (one swizzle atom column)
+constexpr float kRescaleThreshold = 8.0f;    // log2 units
+
+template <int DCH> struct PrefillRing { static constexpr int NST = DCH == 2 ? 4 : 8; };
+
+template <int DCH>
+constexpr size_t prefill_smem_bytes() {
+    return 1024 + size_t(2 + PrefillRing<DCH>::NST) * DCH * kChunkBytes + 512;
+}
+
+struct SlotInfo {
+    int h, q0, n_kv, n_full;
+};
+
+__device__ __forceinline__ SlotInfo prefill_slot(const PrefillParams& p, int h, int qb) {
+    SlotInfo s;
+    s.h = h;
+    s.q0 = qb * 128;
+    if (s.q0 >= p.Tq) {
+        s.n_kv = 0;
+        s.n_full = 0;
+        return s;
+    }
+    const int64_t qlast = min64(s.q0 + 127, p.Tq - 1);
+    const int64_t kv_end = p.causal ? min64(p.S, p.start_pos + qlast + 1) : p.S;
+    s.n_kv = int((kv_end + 127) / 128);
+    const int64_t full_c = p.causal ? (p.start_pos + s.q0 + 1) / 128 : (p.S / 128);
+    s.n_full = int(min64(full_c, p.S / 128));
+    return s;
+}
+
+template <typename T, int DCH>
+__global__ void __launch_bounds__(kPfThreads, 1)
+prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+    constexpr int NST = PrefillRing<DCH>::NST;
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    unsigned char* base_ptr = smem_raw + (base - smem_u32(smem_raw));
+    const uint32_t sQ = base;                                      // [2][DCH] chunks
+    const uint32_t sRing = base + 2 * DCH * kChunkBytes;           // [NST][DCH] chunks
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + (2 + NST) * DCH * kChunkBytes);
+    uint64_t* q_full = bars;            // 2
+    uint64_t* kv_full = bars + 2;       // NST
+    uint64_t* kv_empty = kv_full + NST; // NST
+    uint64_t* s_full = kv_empty + NST;  // 2
+    uint64_t* p_ready = s_full + 2;     // 2
+    uint64_t* o_done = p_ready + 2;     // 2
+    uint64_t* drain = o_done + 2;       // 1
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- work unit (heaviest first)
+    const int level = blockIdx.x / p.units_per_level;
+    const int rem = blockIdx.x % p.units_per_level;
+    int b, kvh;
+    SlotInfo slot[2];
+    if (p.pair_mode == 0) {
+        const int half = p.G / 2;
+        const int qb = p.n_qb - 1 - level;
+        b = rem / (p.Hkv * half);
+        const int r2 = rem % (p.Hkv * half);
+        kvh = r2 / half;
+        const int h0 = kvh * p.G + 2 * (r2 % half);
+        slot[0] = prefill_slot(p, h0, qb);
+        slot[1] = prefill_slot(p, h0 + 1, qb);
+    } else {
+        const int n_levels = (p.n_qb + 1) / 2;
+        const int qbp = n_levels - 1 - level;
+        b = rem / p.H;
+        const int h = rem % p.H;
+        kvh = h / p.G;
+        slot[0] = prefill_slot(p, h, 2 * qbp);
+        slot[1] = prefill_slot(p, h, 2 * qbp + 1);
+    }
+    const int nmax = max(slot[0].n_kv, slot[1].n_kv);
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&q_full[0]), 1);
+        mbar_init(smem_u32(&q_full[1]), 1);
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(smem_u32(&kv_full[i]), 1);
+            mbar_init(smem_u32(&kv_empty[i]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&s_full[s]), 1);
+            mbar_init(smem_u32(&p_ready[s]), 128);
+            mbar_init(smem_u32(&o_done[s]), 1);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            for (int s = 0; s < 2; ++s) {
+                if (slot[s].n_kv == 0) continue;
+                const uint32_t bar = smem_u32(&q_full[s]);
+                mbar_expect_tx(bar, DCH * kChunkBytes);
+                for (int c = 0; c < DCH; ++c)
+                    tma_load_3d(sQ + (s * DCH + c) * kChunkBytes, &tmQ, bar, c * 64, slot[s].q0,
+                                b * p.H + slot[s].h);
+            }
+            const int zkv = b * p.Hkv + kvh;
+            int issued = 0;
+            for (int i = 0; i < 2 * nmax; ++i) {
+                const int st = i % NST;
+                if (!mbar_wait(smem_u32(&kv_empty[st]), ((i / NST) & 1) ^ 1, p.timeout_ns, abort_flag))
+                    break;
+                issued = i + 1;
+                const uint32_t bar = smem_u32(&kv_full[st]);
+                mbar_expect_tx(bar, DCH * kChunkBytes);
+                const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+                for (int c = 0; c < DCH; ++c)
+                    tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64, (i >> 1) * 128,
+                                zkv);
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
+                mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.timeout_ns, nullptr);
+            for (int s = 0; s < 2; ++s)
+                if (slot[s].n_kv > 0) mbar_wait(smem_u32(&q_full[s]), 0, p.timeout_ns, nullptr);
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_f16(kBF16, 128, 128, false);
+            const uint32_t idO = idesc_f16(kBF16, 128, p.d, true);
+            const int nk = p.d / 16;
+            auto issue_S = [&](int s, int st) {
+                for (int kk = 0; kk < nk; ++kk) {
+                    const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+                    const uint64_t a = smem_desc_sw128(sQ + s * DCH * kChunkBytes + off, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(sRing + st * DCH * kChunkBytes + off, 16, 1024);
+                    mma_ss(tmem + s * 128, a, bd, idS, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_PV = [&](int s, int st, bool accumulate) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t bd = smem_desc_sw128(sRing + st * DCH * kChunkBytes + kk * 2048,
+                                                        kChunkBytes, 1024);
+                    mma_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8, bd, idO,
+                           (accumulate || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = true;
+            for (int s = 0; s < 2 && ok; ++s)
+                if (slot[s].n_kv > 0) ok = mbar_wait(smem_u32(&q_full[s]), 0, p.timeout_ns, abort_flag);
+            if (ok) ok = mbar_wait(smem_u32(&kv_full[0]), 0, p.timeout_ns, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                for (int s = 0; s < 2; ++s) {
+                    if (slot[s].n_kv == 0) continue;
+                    issue_S(s, 0);
+                    mma_commit(smem_u32(&s_full[s]));
+                }
+                mma_commit(smem_u32(&kv_empty[0]));
+            }
+            for (int n = 0; n < nmax && ok; ++n) {
+                const int iV = 2 * n + 1, iK = 2 * n + 2;
+                const int stV = iV % NST, stK = iK % NST;
+                const bool nextK = n + 1 < nmax;
+                ok = mbar_wait(smem_u32(&kv_full[stV]), (iV / NST) & 1, p.timeout_ns, abort_flag);
+                if (ok && nextK)
+                    ok = mbar_wait(smem_u32(&kv_full[stK]), (iK / NST) & 1, p.timeout_ns, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                for (int s = 0; s < 2; ++s) {
+                    if (n >= slot[s].n_kv) continue;
+                    if (!mbar_wait(smem_u32(&p_ready[s]), n & 1, p.timeout_ns, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_PV(s, stV, n > 0);
+                    if (n == slot[s].n_kv - 1) mma_commit(smem_u32(&o_done[s]));
+                    if (n + 1 < slot[s].n_kv) {
+                        issue_S(s, stK);
+                        mma_commit(smem_u32(&s_full[s]));
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&kv_empty[stV]));
+                if (nextK) mma_commit(smem_u32(&kv_empty[stK]));
+            }
+            // every MMA issued must finish before TMEM is released
+            mma_commit(smem_u32(drain));
+            mbar_wait(smem_u32(drain), 0, p.timeout_ns, nullptr);
+        }
+    } else if (warp >= 4) {
+        // ================================================= softmax + epilogue
+        const int s = (warp - 4) >> 2;
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const SlotInfo sl = slot[s];
+        if (sl.n_kv > 0) {
+            const uint32_t tS = tmem + (uint32_t(wq * 32) << 16) + s * 128;
+            const uint32_t tO = tmem + (uint32_t(wq * 32) << 16) + 256 + s * 128;
+            const int64_t qpos = p.start_pos + sl.q0 + row;
+            const float c2 = p.scale_log2;
+            float m_run = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int n = 0; n < sl.n_kv; ++n) {
+                ok = mbar_wait(smem_u32(&s_full[s]), n & 1, p.timeout_ns, abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t r0[32], r1[32], r2[32], r3[32];
+                tmem_ld32(tS + 0, r0);
+                tmem_ld32(tS + 32, r1);
+                tmem_ld32(tS + 64, r2);
+                tmem_ld32(tS + 96, r3);
+                tmem_wait_ld();
+                float sv[128];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    sv[c] = __uint_as_float(r0[c]);
+                    sv[32 + c] = __uint_as_float(r1[c]);
+                    sv[64 + c] = __uint_as_float(r2[c]);
+                    sv[96 + c] = __uint_as_float(r3[c]);
+                }
+                if (n >= sl.n_full) {
+                    int64_t lim = p.causal ? qpos - int64_t(n) * 128 : 127;
+                    lim = min64(lim, p.S - 1 - int64_t(n) * 128);
+                    const int li = int(max64(-1, min64(127, lim)));
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c > li) sv[c] = -INFINITY;
+                }
+                float mx = sv[0];
+#pragma unroll
+                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+                const float m_tile = mx * c2;
+                if (n == 0) {
+                    m_run = m_tile;
+                } else {
+                    const bool need = m_tile - m_run > kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, need)) {
+                        const float alpha = need ? ex2(m_run - m_tile) : 1.f;
+                        if (need) {
+                            l *= alpha;
+                            m_run = m_tile;
+                        }
+                        // O_s is final for tile n-1 (its MMA completed before S_s(n))
+                        for (int cc = 0; cc < p.d; cc += 16) {
+                            uint32_t x[16];
+                            tmem_ld16(tO + cc, x);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                x[e] = __float_as_uint(__uint_as_float(x[e]) * alpha);
+                            tmem_st16(tO + cc, x);
+                        }
+                    }
+                }
+                const float neg_m = -m_run;
+                uint32_t pk[32];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float p0 = ex2(fmaf(sv[half * 64 + 2 * c], c2, neg_m));
+                        const float p1 = ex2(fmaf(sv[half * 64 + 2 * c + 1], c2, neg_m));
+                        l += p0 + p1;
+                        pk[c] = pack2<T>(p0, p1);
+                    }
+                    tmem_st32(tS + half * 32, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&p_ready[s]));
+            }
+            // ---- epilogue: O / l, rounded to the output type
+            if (ok) ok = mbar_wait(smem_u32(&o_done[s]), 0, p.timeout_ns, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+                const bool valid = sl.q0 + row < p.Tq;
+                const size_t orow = (size_t(b) * p.H + sl.h) * p.Tq + sl.q0 + row;
+                T* optr = static_cast<T*>(p.o) + orow * p.d;
+                const float inv = 1.f / l;
+                for (int cc = 0; cc < p.d; cc += 16) {
+                    uint32_t x[16];
+                    tmem_ld16(tO + cc, x);
+                    tmem_wait_ld();
+                    uint4 w0, w1;
+                    w0.x = pack2<T>(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv);
+                    w0.y = pack2<T>(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv);
+                    w0.z = pack2<T>(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv);
+                    w0.w = pack2<T>(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv);
+                    w1.x = pack2<T>(__uint_as_float(x[8]) * inv, __uint_as_float(x[9]) * inv);
+                    w1.y = pack2<T>(__uint_as_float(x[10]) * inv, __uint_as_float(x[11]) * inv);
+                    w1.z = pack2<T>(__uint_as_float(x[12]) * inv, __uint_as_float(x[13]) * inv);
+                    w1.w = pack2<T>(__uint_as_float(x[14]) * inv, __uint_as_float(x[15]) * inv);
+                    if (valid) {
+                        reinterpret_cast<uint4*>(optr + cc)[0] = w0;
+                        reinterpret_cast<uint4*>(optr + cc)[1] = w1;
+                    }
+                }
+                if (valid && p.lse) p.lse[orow] = (m_run + log2f(l)) * 0.69314718055994531f;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace b200attn
