@@ -1,0 +1,596 @@
+#!/usr/bin/env python
+"""Benchmark of the causal attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one call of the library on one batch of the workload (default: the
+BitNet-3B-shaped causal MHA prefill, B=1, H=32, T=2048, d=80, bf16).  The
+line also carries the cached-decode half of the metric (GQA decode, B=64,
+H=32/8, S=8192, d=128, bf16) measured the same way, with its own roofline.
+
+Timing: W untimed steps, then exactly K timed steps bracketed by a barrier and
+torch.cuda.synchronize() on both sides.  Before every timed call L2 is flushed
+by writing 256 MiB (> 126 MB L2); each call is bracketed by CUDA events on the
+launching stream, and the per-step time is the mean event duration, max over
+ranks.  Multi-GPU runs are weak scaling: every rank runs the whole workload on
+its own GPU (the path shards by sequence and head with no exchange).
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+this operation here) on the host cores, on bounded row samples of the same
+workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "prefill TFLOP/s & cached-decode HBM GB/s, causal GQA attn, % of B200 roofline"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    # the four 16-bit workloads; the default is the BitNet-3B-shaped prefill
+    "bitnet3b_mha_prefill_bf16": dict(kind="prefill", dtype="bf16", B=1, H=32, Hkv=32, T=2048,
+                                      d=80),
+    "gqa16x8_prefill_bf16": dict(kind="prefill", dtype="bf16", B=8, H=16, Hkv=8, T=4096, d=128),
+    "gqa_decode_bf16": dict(kind="cached", dtype="bf16", B=64, H=32, Hkv=8, Tnew=1, start=8191,
+                            S=8192, d=128),
+    "mqa_chunked_prefill_f16": dict(kind="cached", dtype="f16", B=32, H=8, Hkv=1, Tnew=512,
+                                    start=3584, S=4096, d=128),
+}
+DEFAULT_WORKLOAD = "bitnet3b_mha_prefill_bf16"
+DECODE_WORKLOAD = "gqa_decode_bf16"
+TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
+KERNEL_SOURCES = {"tcgen05": "prefill_tcgen05.cuh", "splitkv": "decode_splitkv.cuh",
+                  "simt": "simt_attn.cuh"}
+
+
+# ------------------------------------------------------------------ workload algebra
+
+def q_len(w):
+    return w["T"] if w["kind"] == "prefill" else w["Tnew"]
+
+
+def kv_len(w):
+    return w["T"] if w["kind"] == "prefill" else w["S"]
+
+
+def start_pos(w):
+    return 0 if w["kind"] == "prefill" else w["start"]
+
+
+def visible_pairs(w):
+    """Visible (query, key) pairs per query head: sum over rows of (p_i + 1)."""
+    Tq, s0 = q_len(w), start_pos(w)
+    return Tq * s0 + Tq * (Tq + 1) // 2
+
+
+def algorithmic_flops(w):
+    """4*d FLOPs per visible (query, key) pair per query head (2*d for Q.K, 2*d
+    for P.V); masked pairs, exponentials and maxima are not counted."""
+    return 4 * w["d"] * w["B"] * w["H"] * visible_pairs(w)
+
+
+def algorithmic_bytes(w):
+    """Q read + the visible K/V rows read once per K/V head + O written."""
+    esz = 2 if w["dtype"] in ("bf16", "f16") else 4
+    kv_vis = min(kv_len(w), start_pos(w) + q_len(w))
+    q_o = 2 * w["B"] * w["H"] * q_len(w) * w["d"] * esz
+    return q_o + 2 * w["B"] * w["Hkv"] * kv_vis * w["d"] * esz
+
+
+def bound(w):
+    return "hbm" if w["kind"] == "cached" and q_len(w) * w["H"] // w["Hkv"] <= 16 else "tensor"
+
+
+def config_of(name, w, world):
+    cfg = {"workload": name, "B": w["B"], "H": w["H"], "Hkv": w["Hkv"], "d": w["d"],
+           "dtype": w["dtype"], "causal": True, "scale": f"1/sqrt({w['d']})"}
+    if w["kind"] == "prefill":
+        cfg["T"] = w["T"]
+    else:
+        cfg.update(Tnew=w["Tnew"], start_pos=w["start"], S=w["S"])
+    cfg["l2"] = "flushed by a 256 MiB write before every timed call"
+    cfg["global_batch"] = w["B"] * world
+    cfg["parallelism"] = f"replicas x{world} (weak scaling, no data-path collective)"
+    return cfg
+
+
+# ------------------------------------------------------------------ peaks, clocks, profiles
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            peaks = json.load(fh)
+        return peaks, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            idx = torch.cuda._get_nvml_device_index(device_index)
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nvml = None
+
+    def _sample(self):
+        n = self._nvml
+        try:
+            mhz = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+            reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:  # noqa: BLE001
+            return
+        self.samples.append((mhz, reasons))
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        reasons = set()
+        for _, mask in self.samples:
+            for bit, name in REASON_BITS.items():
+                if mask & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples)}
+
+
+def clocks_rejected(cl):
+    if cl["sm_mhz"] is None:
+        return False
+    if BAD_REASONS & set(cl["reasons"]):
+        return True
+    # stuck well below max with no reason at all: a leftover clock lock
+    return (cl["sm_max_mhz"] and cl["sm_mhz"] < 0.6 * cl["sm_max_mhz"] and
+            not (set(cl["reasons"]) - {"gpu_idle"}))
+
+
+def kernel_source_sha(kernel: str) -> str:
+    path = os.path.join(ROOT, "transformer_attention_causal_b200", "csrc", KERNEL_SOURCES[kernel])
+    with open(path, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when there is none or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m_bytes or not m_sha or m_sha.group(1) != kernel_source_sha(kernel):
+        return None
+    return float(m_bytes.group(1))
+
+
+# ------------------------------------------------------------------ our implementation
+
+class Case:
+    """Device buffers and the library call for one workload."""
+
+    def __init__(self, name, w, device, seed=0):
+        import transformer_attention_causal_b200 as attn
+        from transformer_attention_causal_b200 import inputs
+
+        self.attn, self.name, self.w = attn, name, w
+        dt = TORCH_DTYPE[w["dtype"]]
+        self.dtype = dt
+        Tq, S = q_len(w), kv_len(w)
+        q, k, v = inputs.qkv(w["B"], w["H"], w["Hkv"], Tq, S, w["d"], dt, seed=seed)
+        self.host = [t.pin_memory() for t in (q, k, v)]
+        self.q, self.k, self.v = (t.to(device, non_blocking=True) for t in self.host)
+        self.out = torch.empty_like(self.q)
+        self.out_host = torch.empty(self.out.shape, dtype=dt).pin_memory()
+        self.scale = 1.0 / math.sqrt(w["d"])
+        if w["kind"] == "prefill":
+            self.kernel = attn.prefill_plan(dt, w["B"], w["H"], w["Hkv"], Tq, w["d"])
+            self.ws = None
+        else:
+            self.kernel = attn.cached_plan(dt, w["B"], w["H"], w["Hkv"], Tq, S, S, w["d"],
+                                           w["start"])
+            need = attn.cached_workspace_size(dt, w["B"], w["H"], w["Hkv"], Tq, S, w["d"],
+                                              w["start"])
+            self.ws = torch.empty(need, dtype=torch.uint8, device=device) if need else None
+        # launches of this library's kernels per call
+        self.launches = 1
+        if self.kernel == "splitkv" and self.ws is not None:
+            self.launches = 2
+
+    def call(self):
+        w = self.w
+        if w["kind"] == "prefill":
+            self.attn.prefill(self.q, self.k, self.v, scale=self.scale, causal=True, out=self.out)
+        else:
+            self.attn.cached(self.q, self.k, self.v, start_pos=w["start"], scale=self.scale,
+                             out=self.out, workspace=self.ws)
+
+
+def time_device(case, steps, warmup, dist_ctx):
+    """Mean per-call device time (ms) over `steps` timed calls, L2 flushed
+    before each; returns (kernel_ms, bracket_ms)."""
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=case.q.device)
+    for _ in range(warmup):
+        flush.zero_()
+        case.call()
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    b0 = torch.cuda.Event(enable_timing=True)
+    b1 = torch.cuda.Event(enable_timing=True)
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    b0.record()
+    for i in range(steps):
+        flush.zero_()
+        ev_s[i].record()
+        case.call()
+        ev_e[i].record()
+    b1.record()
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    kernel_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(steps)) / steps
+    return kernel_ms, b0.elapsed_time(b1)
+
+
+def time_e2e(case, steps, warmup, dist_ctx):
+    """Per-step time (ms) with the inputs copied host -> device from pinned
+    memory and the output copied back, every step."""
+    def step():
+        case.q.copy_(case.host[0], non_blocking=True)
+        case.k.copy_(case.host[1], non_blocking=True)
+        case.v.copy_(case.host[2], non_blocking=True)
+        case.call()
+        case.out_host.copy_(case.out, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    b0 = torch.cuda.Event(enable_timing=True)
+    b1 = torch.cuda.Event(enable_timing=True)
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    b0.record()
+    for _ in range(steps):
+        step()
+    b1.record()
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    h2d = sum(t.numel() * t.element_size() for t in case.host)
+    d2h = case.out_host.numel() * case.out_host.element_size()
+    return b0.elapsed_time(b1) / steps, h2d, d2h
+
+
+class DistCtx:
+    """One process per GPU (torchrun env).  NCCL carries only the barrier and
+    the max-over-ranks of the timings; the data path has no collective.
+    ``backend="gloo"`` runs the same host logic on CPU (tests)."""
+
+    def __init__(self, backend: str = "nccl"):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            kwargs = {}
+            if backend == "nccl":
+                torch.cuda.set_device(self.local_rank)
+                kwargs["device_id"] = torch.device("cuda", self.local_rank)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kwargs)
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def roofline(w, kernel_ms, kernel, name, peaks, peak_src):
+    if bound(w) == "hbm":
+        achieved = algorithmic_bytes(w) / (kernel_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    else:
+        achieved = algorithmic_flops(w) / (kernel_ms * 1e-3) / 1e12
+        # a kernel timed alone: the burst GEMM figure
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    return {"bound": bound(w), "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
+            if peak_src == "measured" else "fallback", "traffic": profiled_traffic(kernel, name),
+            "kernel": kernel}
+
+
+def cpu_baseline(w, name, target_s=10.0):
+    """The fp64 oracle, as it stands, on a bounded seeded row sample of the
+    workload, on every host core."""
+    import numpy as np
+
+    from oracle import attention as oracle_attention
+    from oracle import num_cores
+    from transformer_attention_causal_b200 import inputs
+
+    dt = TORCH_DTYPE[w["dtype"]]
+    Tq, S, s0 = q_len(w), kv_len(w), start_pos(w)
+    q, k, v = inputs.qkv(w["B"], w["H"], w["Hkv"], Tq, S, w["d"], dt, seed=0)
+    total_rows = w["B"] * w["H"] * Tq
+    rng = np.random.default_rng(0)
+
+    def row_flops(rows):
+        i = np.asarray(rows) % Tq
+        return float(np.sum(4 * w["d"] * (s0 + i + 1)))
+
+    def run(n):
+        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+        t0 = time.perf_counter()
+        oracle_attention(q, k, v, scale=1 / math.sqrt(w["d"]), causal=True, start_pos=s0,
+                         rows=rows)
+        return time.perf_counter() - t0, row_flops(rows), len(rows)
+
+    dt_pilot, fl_pilot, _ = run(4 * num_cores())
+    rate = fl_pilot / max(dt_pilot, 1e-6)
+    per_row = algorithmic_flops(w) / total_rows
+    n = int(min(total_rows, max(64, target_s * rate / per_row)))
+    secs, flops, nrows = run(n)
+    if bound(w) == "hbm":
+        esz = 2 if w["dtype"] != "f32" else 4
+        byts = nrows * (2 * w["d"] * esz + 2 * min(S, s0 + Tq) * w["d"] * esz)
+        value, unit = byts / secs / 1e9, "GB/s"
+    else:
+        value, unit = flops / secs / 1e12, "TFLOP/s"
+    return {"value": value, "unit": unit, "cores": num_cores(), "kind": "oracle",
+            "sample": f"{nrows} seeded random rows of {total_rows} ({secs:.1f} s, "
+                      f"fp64 two-pass softmax)"}
+
+
+def whole_job_value(world: int, work_per_step: float, slowest_ms: float) -> float:
+    """Weak scaling: every rank does `work_per_step`; the job is as fast as
+    its slowest rank."""
+    return world * work_per_step / (slowest_ms * 1e-3)
+
+
+def workload(name: str, batch: int | None = None):
+    w = dict(WORKLOADS[name])
+    if batch:
+        w["B"] = int(batch)
+    return w
+
+
+def run_ours(args, dist_ctx):
+    name = args.workload
+    w = workload(name, args.batch)
+    device = torch.device("cuda", dist_ctx.local_rank)
+    torch.cuda.set_device(device)
+    from transformer_attention_causal_b200.build import build
+
+    if dist_ctx.rank == 0:
+        build()
+    dist_ctx.barrier()
+    peaks, peak_src = load_peaks()
+    case = Case(name, w, device)
+    torch.cuda.synchronize()
+
+    def measure():
+        with ClockSampler(device.index) as cs:
+            k_ms, br_ms = time_device(case, args.steps, args.warmup, dist_ctx)
+            e_ms, h2d, d2h = time_e2e(case, args.steps, args.warmup, dist_ctx)
+        return k_ms, br_ms, e_ms, h2d, d2h, cs.summary()
+
+    k_ms, br_ms, e_ms, h2d, d2h, clocks = measure()
+    if clocks_rejected(clocks):
+        k_ms, br_ms, e_ms, h2d, d2h, clocks = measure()
+        clocks["remeasured"] = True
+    k_ms, br_ms, e_ms = dist_ctx.max(k_ms), dist_ctx.max(br_ms), dist_ctx.max(e_ms)
+    from transformer_attention_causal_b200 import device_status
+
+    status = device_status()
+    N = dist_ctx.world
+    unit = "GB/s" if bound(w) == "hbm" else "TFLOP/s"
+    work = algorithmic_bytes(w) / 1e9 if unit == "GB/s" else algorithmic_flops(w) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(whole_job_value(N, work, k_ms), 3),
+        "unit": unit,
+        "n_gpus": N,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(k_ms, 5),
+        "bracket_ms": round(br_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w["dtype"],
+        "data": "synthetic: i.i.d. N(0,1) from seed 0, rounded to the dtype",
+        "config": config_of(name, w, N),
+        "e2e": {"value": round(whole_job_value(N, work, e_ms), 3), "unit": unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": roofline(w, k_ms, case.kernel, name, peaks, peak_src),
+        "gpu_launches": args.steps * case.launches,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if not args.no_decode and name != DECODE_WORKLOAD:
+        del case
+        torch.cuda.empty_cache()
+        wd = WORKLOADS[DECODE_WORKLOAD]
+        dcase = Case(DECODE_WORKLOAD, wd, device)
+        dsteps = max(args.steps, 5)
+        d_ms, _ = time_device(dcase, dsteps, max(args.warmup, 3), dist_ctx)
+        d_ms = dist_ctx.max(d_ms)
+        line["decode"] = {
+            "workload": DECODE_WORKLOAD,
+            "value": round(N * algorithmic_bytes(wd) / 1e9 / (d_ms * 1e-3), 2),
+            "unit": "GB/s", "ms_per_step": round(d_ms, 5), "steps": dsteps,
+            "gpu_launches": dsteps * dcase.launches,
+            "roofline": roofline(wd, d_ms, dcase.kernel, DECODE_WORKLOAD, peaks, peak_src),
+        }
+    if dist_ctx.rank == 0 and N == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, name)
+    if dist_ctx.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, dist_ctx):
+    """The oracle as the reference arm: each step a bounded row sample."""
+    if dist_ctx.rank != 0:
+        return
+    import numpy as np
+
+    from oracle import attention as oracle_attention
+    from oracle import num_cores
+    from transformer_attention_causal_b200 import inputs
+
+    name = args.workload
+    w = workload(name, args.batch)
+    dt = TORCH_DTYPE[w["dtype"]]
+    Tq, S, s0 = q_len(w), kv_len(w), start_pos(w)
+    q, k, v = inputs.qkv(w["B"], w["H"], w["Hkv"], Tq, S, w["d"], dt, seed=0)
+    total_rows = w["B"] * w["H"] * Tq
+    per_step_s = min(5.0, 150.0 / max(1, args.steps + args.warmup))
+    rng = np.random.default_rng(1)
+    unit = "GB/s" if bound(w) == "hbm" else "TFLOP/s"
+    esz = 2 if w["dtype"] != "f32" else 4
+
+    def work_of(rows):
+        i = np.asarray(rows) % Tq
+        if unit == "GB/s":
+            return float(len(rows) * (2 * w["d"] * esz + 2 * min(S, s0 + Tq) * w["d"] * esz)) / 1e9
+        return float(np.sum(4 * w["d"] * (s0 + i + 1))) / 1e12
+
+    def step(n):
+        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+        t0 = time.perf_counter()
+        oracle_attention(q, k, v, scale=1 / math.sqrt(w["d"]), causal=True, start_pos=s0,
+                         rows=rows)
+        return time.perf_counter() - t0, work_of(rows), len(rows)
+
+    secs, work, _ = step(4 * num_cores())
+    per_row = (algorithmic_flops(w) / 1e12 if unit == "TFLOP/s" else algorithmic_bytes(w) / 1e9) \
+        / total_rows
+    n = int(min(total_rows, max(16, per_step_s * (work / max(secs, 1e-6)) / per_row)))
+    for _ in range(args.warmup):
+        step(n)
+    tot_s, tot_w, nrows = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        s_, w_, r_ = step(n)
+        tot_s, tot_w, nrows = tot_s + s_, tot_w + w_, nrows + r_
+    value = tot_w / tot_s
+    line = {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": unit, "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: i.i.d. N(0,1) from seed 0, rounded to the dtype",
+        "config": config_of(name, w, 1),
+        "cpu_baseline": {"value": value, "unit": unit, "cores": num_cores(), "kind": "oracle",
+                         "sample": f"{n} seeded random rows of {total_rows} per step"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode half")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (smaller profiling captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        # no process group: under torchrun the other ranks simply exit
+        run_reference(args, _NoDist())
+        return
+    dist_ctx = DistCtx()
+    try:
+        run_ours(args, dist_ctx)
+    finally:
+        dist_ctx.close()
+
+
+class _NoDist:
+    def __init__(self):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    def barrier(self):
+        pass
+
+
+if __name__ == "__main__":
+    main()

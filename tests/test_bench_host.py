@@ -1,0 +1,89 @@
+"""Host-side logic of bench.py, on the CPU: work accounting, the weak-scaling
+aggregate over ranks (2 gloo ranks), clock-record rejection, and the staleness
+check of committed profile figures."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+
+
+def brute_visible_pairs(Tq, S, start):
+    i = np.arange(Tq)[:, None] + start
+    j = np.arange(S)[None, :]
+    return int((j <= i).sum())
+
+
+@pytest.mark.parametrize("Tq,S,start", [(16, 16, 0), (7, 30, 23), (1, 9, 8), (5, 12, 3)])
+def test_visible_pairs_match_a_mask_count(Tq, S, start):
+    w = dict(kind="cached", Tnew=Tq, S=S, start=start)
+    assert bench.visible_pairs(w) == brute_visible_pairs(Tq, S, start)
+
+
+def test_workload_work_figures():
+    W = bench.WORKLOADS
+    # 4*d FLOPs per visible pair per query head
+    assert bench.algorithmic_flops(W["bitnet3b_mha_prefill_bf16"]) == 4 * 80 * 32 * 2048 * 2049 // 2
+    assert bench.algorithmic_flops(W["gqa16x8_prefill_bf16"]) == 4 * 128 * 8 * 16 * 4096 * 4097 // 2
+    pairs = sum(3584 + i + 1 for i in range(512))
+    assert pairs == 1966336
+    assert bench.algorithmic_flops(W["mqa_chunked_prefill_f16"]) == 4 * 128 * 32 * 8 * pairs
+    # decode: K + V once per K/V head, plus Q and O
+    assert bench.algorithmic_bytes(W["gqa_decode_bf16"]) == 2148532224
+    assert bench.bound(W["gqa_decode_bf16"]) == "hbm"
+    assert bench.bound(W["mqa_chunked_prefill_f16"]) == "tensor"
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    ctx = bench.DistCtx(backend="gloo")
+    ctx.barrier()
+    slowest = ctx.max(1.0 + rank)       # rank 1 is the slow one: 2.0 ms
+    results[rank] = (slowest, bench.whole_job_value(ctx.world, 21.0, slowest))
+    ctx.close()
+
+
+def test_two_ranks_take_the_slowest_rank():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        results = mgr.dict()
+        mp.spawn(_rank_main, args=(world, port, results), nprocs=world, join=True)
+        for rank in range(world):
+            slowest, value = results[rank]
+            assert slowest == 2.0
+            assert value == pytest.approx(2 * 21.0 / 2e-3)
+
+
+def test_clock_records_are_rejected_for_thermal_or_locked_clocks():
+    ok = {"sm_mhz": 1900, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}
+    assert not bench.clocks_rejected(ok)
+    assert bench.clocks_rejected({**ok, "reasons": ["hw_thermal_slowdown"]})
+    assert bench.clocks_rejected({"sm_mhz": 900, "sm_max_mhz": 1965, "reasons": []})
+    assert not bench.clocks_rejected({"sm_mhz": 900, "sm_max_mhz": 1965,
+                                      "reasons": ["sw_power_cap"]})
+
+
+def test_profile_traffic_goes_stale_when_the_kernel_changes(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    csrc = tmp_path / "transformer_attention_causal_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "prefill_tcgen05.cuh").write_text("kernel v1")
+    (tmp_path / "profiles").mkdir()
+    sha = bench.kernel_source_sha("tcgen05")
+    prof = tmp_path / "profiles" / "tcgen05_w.md"
+    prof.write_text(f"dram_bytes_per_launch: 1234\nkernel_source_sha256_16: {sha}\n")
+    assert bench.profiled_traffic("tcgen05", "w") == 1234.0
+    (csrc / "prefill_tcgen05.cuh").write_text("kernel v2")
+    assert bench.profiled_traffic("tcgen05", "w") is None
