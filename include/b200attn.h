@@ -109,6 +109,32 @@ ATTN_API attn_status_t attn_cached(const void* q, const void* k_hist, const void
                           int64_t Tnew, int64_t S, int64_t S_cap, int64_t d, int64_t start_pos,
                           float scale, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * attn_cached without a workspace argument, for callers that may not allocate
+ * device memory themselves: plugins that receive only their input and output
+ * buffers from a host framework owning the allocator, and serving loops that
+ * forbid allocation (and the synchronisation it can bring) once warm.  The
+ * pages have no counterpart to this call; it exists for such callers only.
+ *
+ * Same operation, arguments, layouts and errors as attn_cached minus
+ * `workspace` / `workspace_bytes`.  The split-KV partials go to one
+ * library-owned device array of ATTN_NOALLOC_SCRATCH_BYTES (16 MiB), present
+ * on every GPU that loads the library until the process exits.  A problem
+ * whose attn_cached_workspace_size() exceeds that returns
+ * ATTN_ERR_WORKSPACE and launches nothing.  The call allocates nothing: the
+ * first call on each device looks up the array's device address (with that
+ * device current), so make that first call before any stream capture.  All
+ * calls on a device share the one array and it keeps the last call's data;
+ * calls that can overlap on the GPU (different streams, no ordering between
+ * them) race on it and must be serialised by the caller.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
+ATTN_API attn_status_t attn_cached_noalloc(const void* q, const void* k_hist, const void* v_hist,
+                                           void* o, float* lse, attn_dtype_t dtype, int64_t B,
+                                           int64_t H, int64_t Hkv, int64_t Tnew, int64_t S,
+                                           int64_t S_cap, int64_t d, int64_t start_pos,
+                                           float scale, void* stream);
+
 /* Bytes of workspace attn_cached needs for this problem (0 if none).  Pure
  * host arithmetic; valid without a GPU.  Returns 0 for arguments that
  * attn_cached would reject. */

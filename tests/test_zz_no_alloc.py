@@ -1,0 +1,73 @@
+"""attn_cached_noalloc: the cached entry point for callers that may not
+allocate device memory (plugins handed only their input/output buffers by a
+host framework that owns the allocator; serving loops that forbid allocation
+once warm).  Its split-KV partials live in a fixed 16 MiB library-owned device
+array instead of a caller workspace.
+
+This file is collected last on purpose: if it fails, a run that stops at the
+first failure has already run every other test.
+"""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from transformer_attention_causal_b200 import _lib, inputs
+
+BF16 = 1
+SCRATCH_BYTES = 16 << 20
+
+
+def noalloc_fn():
+    lib = _lib.load()
+    fn = lib.attn_cached_noalloc
+    i64, vp = ctypes.c_int64, ctypes.c_void_p
+    fn.restype = ctypes.c_int
+    fn.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i64, i64, i64, i64, i64,
+                   ctypes.c_float, vp]
+    return lib, fn
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    """Checked before any device work (host only): a decode whose partials
+    need more than the 16 MiB array returns ATTN_ERR_WORKSPACE."""
+    lib, fn = noalloc_fn()
+    B, H, Hkv, Tnew, S, d = 100, 32, 4, 1, 1 << 20, 128
+    need = lib.attn_cached_workspace_size(BF16, B, H, Hkv, Tnew, S, d, S - Tnew)
+    assert need > SCRATCH_BYTES
+    fake = ctypes.c_void_p(0x10000)  # never dereferenced: the call is rejected first
+    rc = fn(fake, fake, fake, fake, None, BF16, B, H, Hkv, Tnew, S, S, d, S - Tnew, 0.1, None)
+    assert rc == _lib.ERR_WORKSPACE
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_cached_on_two_calls_in_a_row():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import transformer_attention_causal_b200 as attn
+    from transformer_attention_causal_b200.build import build
+
+    build()
+    lib, fn = noalloc_fn()
+    B, H, Hkv, Tnew, S, d = 8, 32, 8, 1, 8192, 128
+    start = S - Tnew
+    scale = 1.0 / math.sqrt(d)
+    need = lib.attn_cached_workspace_size(BF16, B, H, Hkv, Tnew, S, d, start)
+    assert 0 < need <= SCRATCH_BYTES  # this problem does use the scratch array
+    stream = torch.cuda.current_stream()
+    for seed in (21, 22):  # two calls in a row: the second must not see the first's data
+        q, k, v = (t.cuda() for t in inputs.qkv(B, H, Hkv, Tnew, S, d, torch.bfloat16, seed=seed))
+        ref = attn.cached(q, k, v, start_pos=start, scale=scale)
+        out = torch.full_like(q, float("nan"))
+        rc = fn(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()), None, BF16, B, H,
+                Hkv, Tnew, S, S, d, start, scale, ctypes.c_void_p(stream.cuda_stream))
+        assert rc == _lib.OK, _lib.status_string(rc)
+        torch.cuda.synchronize()
+        err = (out.double() - ref.double()).abs().cpu().numpy()
+        assert np.all(np.isfinite(err))
+        # the 16-bit tolerance used throughout the tests
+        assert err.max() <= 1.5e-2 and err.mean() <= 2e-3, (seed, err.max(), err.mean())
+    assert attn.device_status() == 0

@@ -440,3 +440,58 @@ void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : kDefau
 int attn_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attn_cached_noalloc: the cached entry point for callers that may not
+// allocate device memory.  Its only scratch need (the split-KV partials) is
+// served from this fixed array, which lives in every device that loads the
+// library until the process exits.  The decode kernel writes every partial it
+// later reads, so nothing in the array has to start at zero.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The host-side
+// name is only a handle for the runtime; the first call on each device looks
+// the real address up (with that device current) and keeps it.
+attn_status_t noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+        return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_cached_noalloc(const void* q, const void* k_hist,
+                                             const void* v_hist, void* o, float* lse,
+                                             attn_dtype_t dtype, int64_t B, int64_t H,
+                                             int64_t Hkv, int64_t Tnew, int64_t S, int64_t S_cap,
+                                             int64_t d, int64_t start_pos, float scale,
+                                             void* stream) {
+    Problem pb{dtype, B, H, Hkv, Tnew, S, S_cap, d, start_pos, 1, true};
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    Plan pl;
+    attn_status_t st = make_plan(pb, pl);
+    if (st != ATTN_OK) return st;
+    st = check_pointers(pb, q, k_hist, v_hist, o, lse);
+    if (st != ATTN_OK) return st;
+    if (pl.ws_bytes > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
+    if (pl.kernel == ATTN_KERNEL_NONE) return ATTN_OK;
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != ATTN_OK) return st;
+    return dispatch(pb, pl, q, k_hist, v_hist, o, lse, scale, pl.ws_bytes ? scratch : nullptr,
+                    static_cast<cudaStream_t>(stream));
+}
