@@ -54,9 +54,94 @@ struct PrefillParams {
     uint64_t timeout_ns;
 };
 
-constexpr int kPfThreads = 384;
+constexpr int kPfThreads = 384;  // 12 warps
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 16-bit columns (one swizzle atom column)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
+// Of every 8 column pairs of an unmasked tile, this many take their
+// exponentials on the FMA pipe (exp2_fma2) instead of MUFU.
+constexpr int kEmuPairsPer8 = 3;
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for two values on the FMA/ALU pipes, relative error <= 1.1e-4 over
+// [-126, 16] (gen_exp2_poly.py): j = nearest integer via the 1.5*2^23
+// addition, f = x - j in [-1/2, 1/2], p(f) a degree-3 fit of 2^f with p(0) = 1,
+// and 2^j applied by adding j << 23 to the bits of p(f).  Inputs below -126
+// are clamped (their weights are < 2^-126 of the row's largest and vanish in
+// the fp32 sums); -inf must not reach this function.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    constexpr float kC1 = 6.932829618e-01f, kC2 = 2.422109693e-01f, kC3 = 5.500890315e-02f;
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+    const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+    const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
+    float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+    q = __ffma2_rn(q, f, make_float2(kC1, kC1));
+    q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Columns past `last` of a 32-column chunk of scores (fp32 bits) become -inf.
+__device__ __forceinline__ void mask_chunk(uint32_t (&r)[32], int last) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+        if (c > last) r[c] = 0xff800000u;  // -inf
+}
+
+// Maximum of a 32-column chunk (fp32 bits): four independent max3 chains.
+__device__ __forceinline__ float chunk_max(const uint32_t (&r)[32]) {
+    float m[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) m[a] = fmax3(__uint_as_float(r[a]), __uint_as_float(r[a + 4]),
+                                             __uint_as_float(r[a + 8]));
+#pragma unroll
+    for (int c = 12; c < 28; c += 8)
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+            m[a] = fmax3(m[a], __uint_as_float(r[c + a]), __uint_as_float(r[c + a + 4]));
+#pragma unroll
+    for (int a = 0; a < 4; ++a) m[a] = fmaxf(m[a], __uint_as_float(r[28 + a]));
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// P = 2^(s*c - m) for a 32-column chunk: the fp32 values replace the scores
+// in r, the 16-bit pairs go to TMEM at `taddr` (16 columns).
+template <typename T>
+__device__ __forceinline__ void exp_chunk(uint32_t (&r)[32], float2 c2v, float2 negm, uint32_t taddr) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                                    c2v, negm);
+        const float p0 = ex2(x.x), p1 = ex2(x.y);
+        r[2 * i] = __float_as_uint(p0);
+        r[2 * i + 1] = __float_as_uint(p1);
+        pk[i] = pack2<T>(p0, p1);
+    }
+    tmem_st16(taddr, pk);
+}
+
+// Sum of a 32-column chunk of fp32 values (bits), four packed partial sums.
+__device__ __forceinline__ float chunk_sum(const uint32_t (&r)[32]) {
+    float2 acc[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) acc[a] = make_float2(__uint_as_float(r[2 * a]), __uint_as_float(r[2 * a + 1]));
+#pragma unroll
+    for (int i = 8; i < 32; i += 8)
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+            acc[a] = __fadd2_rn(acc[a], make_float2(__uint_as_float(r[i + 2 * a]), __uint_as_float(r[i + 2 * a + 1])));
+    const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+    const float2 t = __fadd2_rn(s01, s23);
+    return t.x + t.y;
+}
 
 template <int DCH> struct PrefillRing { static constexpr int NST = DCH == 2 ? 4 : 8; };
 
@@ -103,8 +188,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
     uint64_t* kv_full = bars + 2;       // NST
     uint64_t* kv_empty = kv_full + NST; // NST
     uint64_t* s_full = kv_empty + NST;  // 2
-    uint64_t* p_ready = s_full + 2;     // 2
-    uint64_t* o_done = p_ready + 2;     // 2
+    uint64_t* p_ready = s_full + 2;     // [slot][half]: 4
+    uint64_t* o_done = p_ready + 4;     // 2
     uint64_t* drain = o_done + 2;       // 1
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -146,7 +231,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_u32(&s_full[s]), 1);
-            mbar_init(smem_u32(&p_ready[s]), 128);
+            mbar_init(smem_u32(&p_ready[2 * s]), 4);      // one arrive per softmax warp
+            mbar_init(smem_u32(&p_ready[2 * s + 1]), 4);
             mbar_init(smem_u32(&o_done[s]), 1);
         }
         mbar_init(smem_u32(drain), 1);
@@ -210,9 +296,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     mma_ss(tmem + s * 128, a, bd, idS, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_PV = [&](int s, int st, bool accumulate) {
+            auto issue_PV = [&](int s, int st, bool accumulate, int k0) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = k0; kk < k0 + 4; ++kk) {
                     const uint64_t bd = smem_desc_sw128(sRing + st * DCH * kChunkBytes + kk * 2048,
                                                         kChunkBytes, 1024);
                     mma_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8, bd, idO,
@@ -243,12 +329,20 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tc_fence_after();
                 for (int s = 0; s < 2; ++s) {
                     if (n >= slot[s].n_kv) continue;
-                    if (!mbar_wait(smem_u32(&p_ready[s]), n & 1, p.timeout_ns, abort_flag)) {
+                    // P in two halves: the first 64 keys' MMAs start while the
+                    // softmax is still producing the second half
+                    if (!mbar_wait(smem_u32(&p_ready[2 * s]), n & 1, p.timeout_ns, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    issue_PV(s, stV, n > 0);
+                    issue_PV(s, stV, n > 0, 0);
+                    if (!mbar_wait(smem_u32(&p_ready[2 * s + 1]), n & 1, p.timeout_ns, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_PV(s, stV, true, 4);
                     if (n == slot[s].n_kv - 1) mma_commit(smem_u32(&o_done[s]));
                     if (n + 1 < slot[s].n_kv) {
                         issue_S(s, stK);
@@ -265,6 +359,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
     } else if (warp >= 4) {
         // ================================================= softmax + epilogue
+        // warps 4-7: slot 0, warps 8-11: slot 1; one thread per row (TMEM lane).
         const int s = (warp - 4) >> 2;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
@@ -281,32 +376,26 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
+                // All 128 scores of this row in registers (one wait: TMEM
+                // loads are cheap next to the arithmetic that follows).
                 uint32_t r0[32], r1[32], r2[32], r3[32];
                 tmem_ld32(tS + 0, r0);
                 tmem_ld32(tS + 32, r1);
                 tmem_ld32(tS + 64, r2);
                 tmem_ld32(tS + 96, r3);
                 tmem_wait_ld();
-                float sv[128];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    sv[c] = __uint_as_float(r0[c]);
-                    sv[32 + c] = __uint_as_float(r1[c]);
-                    sv[64 + c] = __uint_as_float(r2[c]);
-                    sv[96 + c] = __uint_as_float(r3[c]);
-                }
-                if (n >= sl.n_full) {
+                const bool masked = n >= sl.n_full;
+                if (masked) {
                     int64_t lim = p.causal ? qpos - int64_t(n) * 128 : 127;
                     lim = min64(lim, p.S - 1 - int64_t(n) * 128);
                     const int li = int(max64(-1, min64(127, lim)));
-#pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (c > li) sv[c] = -INFINITY;
+                    mask_chunk(r0, li);
+                    mask_chunk(r1, li - 32);
+                    mask_chunk(r2, li - 64);
+                    mask_chunk(r3, li - 96);
                 }
-                float mx = sv[0];
-#pragma unroll
-                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
-                const float m_tile = mx * c2;
+                const float m_tile =
+                    fmaxf(fmaxf(chunk_max(r0), chunk_max(r1)), fmaxf(chunk_max(r2), chunk_max(r3))) * c2;
                 if (n == 0) {
                     m_run = m_tile;
                 } else {
@@ -329,22 +418,25 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                         }
                     }
                 }
-                const float neg_m = -m_run;
-                uint32_t pk[32];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float p0 = ex2(fmaf(sv[half * 64 + 2 * c], c2, neg_m));
-                        const float p1 = ex2(fmaf(sv[half * 64 + 2 * c + 1], c2, neg_m));
-                        l += p0 + p1;
-                        pk[c] = pack2<T>(p0, p1);
-                    }
-                    tmem_st32(tS + half * 32, pk);
-                }
+                // P = 2^(S*c - m) per 32-column chunk, packed to 16-bit pairs and
+                // stored at once; the first 64 keys are released to the MMA
+                // before the last 64 are computed.  r* then hold P in fp32.
+                const float2 c2v = make_float2(c2, c2);
+                const float2 negm = make_float2(-m_run, -m_run);
+                exp_chunk<T>(r0, c2v, negm, tS + 0);
+                exp_chunk<T>(r1, c2v, negm, tS + 16);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(smem_u32(&p_ready[s]));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&p_ready[2 * s]));
+                exp_chunk<T>(r2, c2v, negm, tS + 32);
+                exp_chunk<T>(r3, c2v, negm, tS + 48);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&p_ready[2 * s + 1]));
+                // row sum, off the MMA's critical path
+                l += chunk_sum(r0) + chunk_sum(r1) + chunk_sum(r2) + chunk_sum(r3);
             }
             // ---- epilogue: O / l, rounded to the output type
             if (ok) ok = mbar_wait(smem_u32(&o_done[s]), 0, p.timeout_ns, abort_flag);
