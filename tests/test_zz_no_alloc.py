@@ -34,9 +34,19 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     """Checked before any device work (host only): a decode whose partials
     need more than the 16 MiB array returns ATTN_ERR_WORKSPACE."""
     lib, fn = noalloc_fn()
-    B, H, Hkv, Tnew, S, d = 100, 32, 4, 1, 1 << 20, 128
-    need = lib.attn_cached_workspace_size(BF16, B, H, Hkv, Tnew, S, d, S - Tnew)
-    assert need > SCRATCH_BYTES
+    # the split plan decides the partials' size: search for a decode that needs more
+    S = 1 << 20
+    found = None
+    for d, H, Hkv, Tnew in ((128, 32, 4, 1), (128, 16, 2, 1), (256, 16, 4, 1), (64, 32, 4, 2)):
+        for B in (20, 37, 50, 74, 100, 150, 200, 300):
+            need = lib.attn_cached_workspace_size(BF16, B, H, Hkv, Tnew, S, d, S - Tnew)
+            if need > SCRATCH_BYTES:
+                found = (B, H, Hkv, Tnew, d)
+                break
+        if found:
+            break
+    assert found, "no decode shape found whose partials exceed the scratch array"
+    B, H, Hkv, Tnew, d = found
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: the call is rejected first
     rc = fn(fake, fake, fake, fake, None, BF16, B, H, Hkv, Tnew, S, S, d, S - Tnew, 0.1, None)
     assert rc == _lib.ERR_WORKSPACE

@@ -23,10 +23,10 @@ namespace {
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 
-// Planning constants for B200: 148 SMs, two decode CTAs resident per SM.
+// Planning constants for B200: 148 SMs.  The wide decode kernel runs one
+// 512-thread CTA per SM with 120-key stages; the compact one (large row
+// counts) two 160-thread CTAs per SM with 64-key stages.
 constexpr int kPlanSMs = 148;
-constexpr int kDecodeCtasPerSM = 2;
-constexpr int kDecodeStageKeys = 64;
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
@@ -43,6 +43,7 @@ struct Plan {
     attn_kernel_t kernel = ATTN_KERNEL_NONE;
     // split-KV decode
     int R = 0, Rv = 0, nsplit = 1;
+    bool wide = false;
     int64_t chunk = 0, kv_end = 0;
     size_t ws_bytes = 0;
     // tcgen05 prefill
@@ -84,10 +85,13 @@ void plan_decode(const Problem& pb, Plan& pl) {
     const int64_t G = pb.H / pb.Hkv;
     pl.Rv = int(G * pb.Tq);
     pl.R = next_pow2_at_least4(pl.Rv);
+    pl.wide = (pl.R <= 8 && (pb.d == 64 || pb.d == 128)) || (pl.R == 4 && pb.d == 256);
+    const int stage_keys = pl.wide ? 120 : 64;
+    const int ctas_per_sm = pl.wide ? 1 : 2;
     pl.kv_end = std::min<int64_t>(pb.S, pb.start_pos + pb.Tq);
-    const int64_t tiles = (pl.kv_end + kDecodeStageKeys - 1) / kDecodeStageKeys;
+    const int64_t tiles = (pl.kv_end + stage_keys - 1) / stage_keys;
     const int64_t units = pb.B * pb.Hkv;
-    const int64_t slots = int64_t(kPlanSMs) * kDecodeCtasPerSM;
+    const int64_t slots = int64_t(kPlanSMs) * ctas_per_sm;
     // Pick the split count that fills the last wave of CTAs best; prefer fewer
     // splits on ties and keep at least 4 stages per split when there is room.
     int best_n = 1;
@@ -109,7 +113,7 @@ void plan_decode(const Problem& pb, Plan& pl) {
     }
     const int64_t per = (tiles + best_n - 1) / best_n;
     pl.nsplit = best_n;
-    pl.chunk = per * kDecodeStageKeys;
+    pl.chunk = per * stage_keys;
     pl.ws_bytes = 0;
     if (pl.nsplit > 1) {
         const size_t rows = size_t(units) * pl.nsplit * pl.Rv;
@@ -239,8 +243,35 @@ attn_status_t launch_decode_R(const DecodeParams& dp, cudaStream_t stream) {
     return ATTN_OK;
 }
 
+template <typename T, int D, int R>
+attn_status_t launch_decode_wide_R(const DecodeParams& dp, cudaStream_t stream) {
+    constexpr size_t smem = WideShape<D, R>::smem_bytes(sizeof(T));
+    auto kern = decode_wide_kernel<T, D, R>;
+    static std::once_flag once[8];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    attn_status_t st = ATTN_OK;
+    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
+    if (st != ATTN_OK) return st;
+    dim3 grid(unsigned(dp.nsplit), unsigned(dp.B * dp.Hkv));
+    kern<<<grid, 512, smem, stream>>>(dp);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
+    if (dp.nsplit > 1) {
+        const int64_t rows = int64_t(dp.B) * dp.Hkv * dp.Rv;
+        decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, stream>>>(dp);
+        return launch_status();
+    }
+    return ATTN_OK;
+}
+
 template <typename T, int D>
-attn_status_t launch_decode_D(int R, const DecodeParams& dp, cudaStream_t stream) {
+attn_status_t launch_decode_D(int R, bool wide, const DecodeParams& dp, cudaStream_t stream) {
+    if (wide) {
+        if (R == 4) return launch_decode_wide_R<T, D, 4>(dp, stream);
+        if constexpr (D <= 128)
+            if (R == 8) return launch_decode_wide_R<T, D, 8>(dp, stream);
+        return ATTN_ERR_UNSUPPORTED;
+    }
     switch (R) {
     case 4: return launch_decode_R<T, D, 4>(dp, stream);
     case 8: return launch_decode_R<T, D, 8>(dp, stream);
@@ -269,9 +300,9 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
     dp.scale_log2 = scale * 1.4426950408889634f;
     dp.timeout_ns = g_timeout_ns.load();
     switch (pb.d) {
-    case 64: return launch_decode_D<T, 64>(pl.R, dp, stream);
-    case 128: return launch_decode_D<T, 128>(pl.R, dp, stream);
-    case 256: return launch_decode_D<T, 256>(pl.R, dp, stream);
+    case 64: return launch_decode_D<T, 64>(pl.R, pl.wide, dp, stream);
+    case 128: return launch_decode_D<T, 128>(pl.R, pl.wide, dp, stream);
+    case 256: return launch_decode_D<T, 256>(pl.R, pl.wide, dp, stream);
     default: return ATTN_ERR_UNSUPPORTED;
     }
 }

@@ -440,3 +440,327 @@ decode_combine_kernel(const DecodeParams p) {
 }
 
 }  // namespace b200attn
+
+namespace b200attn {
+
+// ---------------------------------------------------------------------------
+// Wide split-KV decode: the same per-warp algorithm as decode_splitkv_kernel,
+// shaped for occupancy.  15 consumer warps + 1 producer warp per CTA (four
+// warps on every SM sub-partition, <= 128 registers each), 120-key stages
+// (8 keys per consumer warp), and every lane handles one 16-byte piece of a
+// key row (8 elements), so a key is split over D/8 lanes and the queries and
+// partial outputs each take R x 8 registers.  Dot products and the weighted
+// sum use packed fp32x2 FMAs.
+template <int D, int R>
+struct WideShape {
+    static constexpr int NW = 15;                      // consumer warps
+    static constexpr int KW = 8;                       // keys per warp per stage
+    static constexpr int TK = NW * KW;                 // keys per stage
+    static constexpr int NST = 3;                      // ring depth
+    static constexpr int E = (R <= 4) ? 8 : 4;         // elements per lane per key
+    static constexpr int LPK = D / E;                  // lanes per key
+    static constexpr int KPG = 32 / LPK;               // keys per warp-wide group
+    static constexpr int GPW = KW / KPG;               // groups per warp per stage
+    static constexpr int LPR = 32 / R;                 // lanes per row in the softmax step
+    static constexpr int SPL = KW / LPR;               // scores per lane in that step
+    static_assert(LPK >= 8 && LPK <= 32 && 32 % LPK == 0, "lanes per key");
+    static_assert(R <= LPK && KW % KPG == 0 && KW % LPR == 0 && SPL >= 1, "split");
+    static constexpr size_t smem_bytes(size_t esz) {
+        return 2 * NST * size_t(TK) * D * esz + size_t(NW) * KW * R * 4 + size_t(NW) * R * 4 +
+               (2 * NST + 2) * 8 + 64;
+    }
+};
+
+template <typename T, int E>
+__device__ __forceinline__ void load_piece(const T* src, float (&f)[E]) {
+    if constexpr (E == 8) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src);
+        const float2 a = unpack2<T>(w.x), b = unpack2<T>(w.y), c = unpack2<T>(w.z), d = unpack2<T>(w.w);
+        f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+    } else {
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        const float2 a = unpack2<T>(w.x), b = unpack2<T>(w.y);
+        f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    }
+}
+
+template <typename T, int D, int R>
+__global__ void __launch_bounds__(512, 1)
+decode_wide_kernel(const DecodeParams p) {
+    using Sh = WideShape<D, R>;
+    constexpr int NW = Sh::NW, TK = Sh::TK, NST = Sh::NST, KW = Sh::KW, E = Sh::E, LPK = Sh::LPK,
+                  KPG = Sh::KPG, GPW = Sh::GPW, LPR = Sh::LPR, SPL = Sh::SPL;
+    extern __shared__ __align__(128) unsigned char smem[];
+    T* ks = reinterpret_cast<T*>(smem);                              // [NST][TK][D]
+    T* vs = ks + size_t(NST) * TK * D;                               // [NST][TK][D]
+    float* sc = reinterpret_cast<float*>(vs + size_t(NST) * TK * D); // [NW][KW][R]
+    float* al = sc + NW * KW * R;                                    // [NW][R]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(al + NW * R);       // full[NST], empty[NST]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * NST);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int unit = blockIdx.y;
+    const int split = blockIdx.x;
+    const int b = unit / p.Hkv;
+    const int kvh = unit % p.Hkv;
+    const int64_t k_begin = int64_t(split) * p.chunk;
+    const int64_t k_end = min64(p.kv_end, k_begin + p.chunk);
+    const int nstages = k_end > k_begin ? int((k_end - k_begin + TK - 1) / TK) : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(smem_u32(&bars[s]), 1);
+            mbar_init(smem_u32(&bars[NST + s]), NW);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const T* kg = static_cast<const T*>(p.k) + (size_t(unit) * p.S_cap) * D;
+    const T* vg = static_cast<const T*>(p.v) + (size_t(unit) * p.S_cap) * D;
+
+    if (warp == NW) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int it = 0; it < nstages; ++it) {
+                const int st = it % NST;
+                if (!mbar_wait(smem_u32(&bars[NST + st]), ((it / NST) & 1) ^ 1, p.timeout_ns, abort_flag))
+                    break;
+                issued = it + 1;
+                const int64_t k0 = k_begin + int64_t(it) * TK;
+                const int n = int(min64(TK, k_end - k0));
+                const uint32_t bytes = uint32_t(n) * D * sizeof(T);
+                const uint32_t full = smem_u32(&bars[st]);
+                mbar_expect_tx(full, 2 * bytes);
+                bulk_load(smem_u32(ks + size_t(st) * TK * D), kg + k0 * D, bytes, full);
+                bulk_load(smem_u32(vs + size_t(st) * TK * D), vg + k0 * D, bytes, full);
+            }
+            for (int it = issued - 1; it >= 0 && it >= issued - NST; --it)
+                mbar_wait(smem_u32(&bars[it % NST]), (it / NST) & 1, p.timeout_ns, nullptr);
+        }
+        return;
+    }
+
+    const int sub = lane % LPK;
+    const int kslot = lane / LPK;
+    const int my_row = sub / (LPK / R);
+    const int e0 = sub * E;  // this lane's elements of every key row
+
+    // queries pre-scaled into the log2 domain, as fp32 pairs
+    float2 q2[R][E / 2];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const bool valid = r < p.Rv;
+        const int g = valid ? r / p.Tnew : 0;
+        const int t = valid ? r % p.Tnew : 0;
+        const T* qrow = static_cast<const T*>(p.q) +
+                        ((size_t(b) * p.H + size_t(kvh) * p.G + g) * p.Tnew + t) * D;
+        float f[E];
+        load_piece<T, E>(qrow + e0, f);
+#pragma unroll
+        for (int j = 0; j < E / 2; ++j)
+            q2[r][j] = valid ? make_float2(f[2 * j] * p.scale_log2, f[2 * j + 1] * p.scale_log2)
+                             : make_float2(0.f, 0.f);
+    }
+    int64_t row_lim[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) row_lim[r] = (r < p.Rv) ? p.start_pos + (r % p.Tnew) : -1;
+
+    float2 o2[R][E / 2];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int j = 0; j < E / 2; ++j) o2[r][j] = make_float2(0.f, 0.f);
+    const int rb = lane / LPR;
+    float m_run = -INFINITY, l_part = 0.f;
+    float* scw = sc + warp * KW * R;
+    float* alw = al + warp * R;
+
+    for (int it = 0; it < nstages; ++it) {
+        const int st = it % NST;
+        if (!mbar_wait(smem_u32(&bars[st]), (it / NST) & 1, p.timeout_ns, abort_flag)) break;
+        const int64_t k0 = k_begin + int64_t(it) * TK;
+        const int nvalid = int(min64(TK, k_end - k0));
+        const T* kst = ks + size_t(st) * TK * D;
+        const T* vst = vs + size_t(st) * TK * D;
+
+        // A. scores
+#pragma unroll
+        for (int gi = 0; gi < GPW; ++gi) {
+            const int kw = gi * KPG + kslot;
+            const int ki = warp * KW + kw;
+            float f[E];
+            load_piece<T, E>(kst + size_t(ki) * D + e0, f);
+            float acc[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float2 a2 = __fmul2_rn(q2[r][0], make_float2(f[0], f[1]));
+#pragma unroll
+                for (int j = 1; j < E / 2; ++j) a2 = __ffma2_rn(q2[r][j], make_float2(f[2 * j], f[2 * j + 1]), a2);
+                acc[r] = a2.x + a2.y;
+            }
+            int n = R;
+#pragma unroll
+            for (int o = LPK / 2; o >= 1; o >>= 1) {
+                if (n > 1) {
+                    const bool upper = (lane & o) != 0;
+#pragma unroll
+                    for (int i = 0; i < R / 2; ++i) {
+                        if (i < n / 2) {
+                            const float send = upper ? acc[i] : acc[i + n / 2];
+                            const float keep = upper ? acc[i + n / 2] : acc[i];
+                            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                        }
+                    }
+                    n >>= 1;
+                } else {
+                    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
+                }
+            }
+            const int64_t j = k0 + ki;
+            bool vis = ki < nvalid;
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                if (r == my_row) vis = vis && (j <= row_lim[r]);
+            if (sub % (LPK / R) == 0) scw[kw * R + my_row] = vis ? acc[0] : -INFINITY;
+        }
+        __syncwarp();
+
+        // B. online softmax over the warp's KW keys, row rb
+        {
+            float s[SPL];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < SPL; ++e) {
+                s[e] = scw[((lane % LPR) * SPL + e) * R + rb];
+                mx = fmaxf(mx, s[e]);
+            }
+#pragma unroll
+            for (int o = LPR / 2; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float m_new = fmaxf(m_run, mx);
+            float alpha = 1.f, psum = 0.f;
+            if (m_new != -INFINITY) {
+                alpha = ex2(m_run - m_new);
+#pragma unroll
+                for (int e = 0; e < SPL; ++e) {
+                    s[e] = ex2(s[e] - m_new);
+                    psum += s[e];
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < SPL; ++e) s[e] = 0.f;
+            }
+            l_part = l_part * alpha + psum;
+            m_run = m_new;
+#pragma unroll
+            for (int e = 0; e < SPL; ++e) scw[((lane % LPR) * SPL + e) * R + rb] = s[e];
+            if (lane % LPR == 0) alw[rb] = alpha;
+        }
+        __syncwarp();
+
+        // C. rescale and accumulate P V
+        {
+            float a[R];
+            bool any = false;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                a[r] = alw[r];
+                any |= (a[r] != 1.f);
+            }
+            if (any) {
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < E / 2; ++jj) o2[r][jj] = __fmul2_rn(o2[r][jj], make_float2(a[r], a[r]));
+            }
+#pragma unroll
+            for (int gi = 0; gi < GPW; ++gi) {
+                const int kw = gi * KPG + kslot;
+                const int ki = warp * KW + kw;
+                if (ki < nvalid) {
+                    float pr[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) pr[r] = scw[kw * R + r];
+                    float f[E];
+                    load_piece<T, E>(vst + size_t(ki) * D + e0, f);
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+#pragma unroll
+                        for (int jj = 0; jj < E / 2; ++jj)
+                            o2[r][jj] = __ffma2_rn(make_float2(pr[r], pr[r]),
+                                                   make_float2(f[2 * jj], f[2 * jj + 1]), o2[r][jj]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars[NST + st]));
+    }
+
+    // ---- merge: key slots of a warp, then the warps of the CTA
+#pragma unroll
+    for (int o = LPK; o < 32; o <<= 1)
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int jj = 0; jj < E / 2; ++jj) {
+                o2[r][jj].x += __shfl_xor_sync(0xffffffffu, o2[r][jj].x, o);
+                o2[r][jj].y += __shfl_xor_sync(0xffffffffu, o2[r][jj].y, o);
+            }
+#pragma unroll
+    for (int o = LPR / 2; o >= 1; o >>= 1) l_part += __shfl_xor_sync(0xffffffffu, l_part, o);
+
+    asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
+    float* mo = reinterpret_cast<float*>(smem);  // [NW][R]
+    float* lo = mo + NW * R;                     // [NW][R]
+    float* oo = lo + NW * R;                     // [NW][R][D]
+    if (lane % LPR == 0) {
+        mo[warp * R + rb] = m_run;
+        lo[warp * R + rb] = l_part;
+    }
+    if (kslot == 0) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int jj = 0; jj < E / 2; ++jj) {
+                oo[(warp * R + r) * D + e0 + 2 * jj] = o2[r][jj].x;
+                oo[(warp * R + r) * D + e0 + 2 * jj + 1] = o2[r][jj].y;
+            }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
+
+    const bool aborted = *abort_flag != 0;
+    for (int idx = threadIdx.x; idx < p.Rv * D; idx += NW * 32) {
+        const int r = idx / D, e = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, mo[w * R + r]);
+        float L = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float f = ex2(mo[w * R + r] - M);
+                L += f * lo[w * R + r];
+                acc += f * oo[(w * R + r) * D + e];
+            }
+        }
+        if (aborted) continue;
+        if (p.nsplit == 1) {
+            const int g = r / p.Tnew, t = r % p.Tnew;
+            const size_t orow = (size_t(b) * p.H + size_t(kvh) * p.G + g) * p.Tnew + t;
+            static_cast<T*>(p.o)[orow * D + e] = from_f32<T>(L > 0.f ? acc / L : 0.f);
+            if (e == 0 && p.lse)
+                p.lse[orow] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+        } else {
+            const size_t pi = (size_t(unit) * p.nsplit + split) * p.Rv + r;
+            p.ws_o[pi * D + e] = acc;
+            if (e == 0) {
+                p.ws_m[pi] = M;
+                p.ws_l[pi] = L;
+            }
+        }
+    }
+}
+
+}  // namespace b200attn
