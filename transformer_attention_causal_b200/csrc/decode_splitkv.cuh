@@ -444,26 +444,33 @@ decode_combine_kernel(const DecodeParams p) {
 namespace b200attn {
 
 // ---------------------------------------------------------------------------
-// Wide split-KV decode: the same per-warp algorithm as decode_splitkv_kernel,
-// shaped for occupancy.  15 consumer warps + 1 producer warp per CTA (four
-// warps on every SM sub-partition, <= 128 registers each), 120-key stages
-// (8 keys per consumer warp), and every lane handles one 16-byte piece of a
-// key row (8 elements), so a key is split over D/8 lanes and the queries and
-// partial outputs each take R x 8 registers.  Dot products and the weighted
-// sum use packed fp32x2 FMAs.
+// Wide split-KV decode: the same online-softmax split as
+// decode_splitkv_kernel, shaped for occupancy and instruction count.
+// 15 consumer warps + 1 producer warp per CTA (four warps on every SM
+// sub-partition, <= 128 registers each), 120-key stages (8 keys per consumer
+// warp).  Scores: a key row is split over LPK = D / EA lanes (EA elements =
+// one or two 16-byte pieces each, chosen so the pre-scaled queries take
+// R x EA = 64 registers), dot products in packed fp32x2 FMAs, one halving
+// shuffle reduction per group of 32 / LPK keys.  Weighted sum: all 32 lanes
+// split the head dimension (EC = D / 32 elements each) and walk the warp's
+// keys, so every lane holds only R x EC partial outputs.
 template <int D, int R>
 struct WideShape {
     static constexpr int NW = 15;                      // consumer warps
     static constexpr int KW = 8;                       // keys per warp per stage
     static constexpr int TK = NW * KW;                 // keys per stage
     static constexpr int NST = 3;                      // ring depth
-    static constexpr int E = (R <= 4) ? 8 : 4;         // elements per lane per key
-    static constexpr int LPK = D / E;                  // lanes per key
+    static constexpr int EA0 = 64 / R;
+    static constexpr int EA = EA0 > D / 8 ? D / 8 : EA0;  // score elements per lane
+    static constexpr int LPK = D / EA;                 // lanes per key (scores)
     static constexpr int KPG = 32 / LPK;               // keys per warp-wide group
     static constexpr int GPW = KW / KPG;               // groups per warp per stage
+    static constexpr int EC = D / 32;                  // weighted-sum elements per lane
     static constexpr int LPR = 32 / R;                 // lanes per row in the softmax step
     static constexpr int SPL = KW / LPR;               // scores per lane in that step
+    static_assert(EA % 8 == 0 || EA == 4, "score pieces are 8 or 16 bytes");
     static_assert(LPK >= 8 && LPK <= 32 && 32 % LPK == 0, "lanes per key");
+    static_assert(EC == 2 || EC == 4 || EC == 8, "weighted-sum piece");
     static_assert(R <= LPK && KW % KPG == 0 && KW % LPR == 0 && SPL >= 1, "split");
     static constexpr size_t smem_bytes(size_t esz) {
         return 2 * NST * size_t(TK) * D * esz + size_t(NW) * KW * R * 4 + size_t(NW) * R * 4 +
@@ -471,16 +478,35 @@ struct WideShape {
     }
 };
 
-template <typename T, int E>
-__device__ __forceinline__ void load_piece(const T* src, float (&f)[E]) {
-    if constexpr (E == 8) {
-        const uint4 w = *reinterpret_cast<const uint4*>(src);
-        const float2 a = unpack2<T>(w.x), b = unpack2<T>(w.y), c = unpack2<T>(w.z), d = unpack2<T>(w.w);
-        f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
-    } else {
-        const uint2 w = *reinterpret_cast<const uint2*>(src);
-        const float2 a = unpack2<T>(w.x), b = unpack2<T>(w.y);
+// n consecutive 16-bit elements (n = 2, 4, 8 or 16) widened to fp32.
+template <typename T, int N>
+__device__ __forceinline__ void load_elems(const T* src, float (&f)[N]) {
+    if constexpr (N == 16) {
+        const uint4 w0 = reinterpret_cast<const uint4*>(src)[0];
+        const uint4 w1 = reinterpret_cast<const uint4*>(src)[1];
+        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 v = unpack2<T>(w[i]);
+            f[2 * i] = v.x;
+            f[2 * i + 1] = v.y;
+        }
+    } else if constexpr (N == 8) {
+        const uint4 w0 = *reinterpret_cast<const uint4*>(src);
+        const uint32_t w[4] = {w0.x, w0.y, w0.z, w0.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 v = unpack2<T>(w[i]);
+            f[2 * i] = v.x;
+            f[2 * i + 1] = v.y;
+        }
+    } else if constexpr (N == 4) {
+        const uint2 w0 = *reinterpret_cast<const uint2*>(src);
+        const float2 a = unpack2<T>(w0.x), b = unpack2<T>(w0.y);
         f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    } else {
+        const float2 a = unpack2<T>(*reinterpret_cast<const uint32_t*>(src));
+        f[0] = a.x; f[1] = a.y;
     }
 }
 
@@ -488,8 +514,8 @@ template <typename T, int D, int R>
 __global__ void __launch_bounds__(512, 1)
 decode_wide_kernel(const DecodeParams p) {
     using Sh = WideShape<D, R>;
-    constexpr int NW = Sh::NW, TK = Sh::TK, NST = Sh::NST, KW = Sh::KW, E = Sh::E, LPK = Sh::LPK,
-                  KPG = Sh::KPG, GPW = Sh::GPW, LPR = Sh::LPR, SPL = Sh::SPL;
+    constexpr int NW = Sh::NW, TK = Sh::TK, NST = Sh::NST, KW = Sh::KW, EA = Sh::EA, LPK = Sh::LPK,
+                  KPG = Sh::KPG, GPW = Sh::GPW, EC = Sh::EC, LPR = Sh::LPR, SPL = Sh::SPL;
     extern __shared__ __align__(128) unsigned char smem[];
     T* ks = reinterpret_cast<T*>(smem);                              // [NST][TK][D]
     T* vs = ks + size_t(NST) * TK * D;                               // [NST][TK][D]
@@ -546,10 +572,12 @@ decode_wide_kernel(const DecodeParams p) {
     const int sub = lane % LPK;
     const int kslot = lane / LPK;
     const int my_row = sub / (LPK / R);
-    const int e0 = sub * E;  // this lane's elements of every key row
+    // score pieces: EA elements per lane, split into 16-byte pieces spread
+    // LPK * 8 elements apart (conflict-free quarter-warp reads)
+    constexpr int NPC = EA >= 8 ? EA / 8 : 1;          // pieces per lane
+    constexpr int PE = EA >= 8 ? 8 : EA;               // elements per piece
 
-    // queries pre-scaled into the log2 domain, as fp32 pairs
-    float2 q2[R][E / 2];
+    float2 q2[R][EA / 2];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const bool valid = r < p.Rv;
@@ -557,22 +585,27 @@ decode_wide_kernel(const DecodeParams p) {
         const int t = valid ? r % p.Tnew : 0;
         const T* qrow = static_cast<const T*>(p.q) +
                         ((size_t(b) * p.H + size_t(kvh) * p.G + g) * p.Tnew + t) * D;
-        float f[E];
-        load_piece<T, E>(qrow + e0, f);
 #pragma unroll
-        for (int j = 0; j < E / 2; ++j)
-            q2[r][j] = valid ? make_float2(f[2 * j] * p.scale_log2, f[2 * j + 1] * p.scale_log2)
-                             : make_float2(0.f, 0.f);
+        for (int c = 0; c < NPC; ++c) {
+            float f[PE];
+            load_elems<T, PE>(qrow + (c * LPK + sub) * PE, f);
+#pragma unroll
+            for (int j = 0; j < PE / 2; ++j)
+                q2[r][c * (PE / 2) + j] =
+                    valid ? make_float2(f[2 * j] * p.scale_log2, f[2 * j + 1] * p.scale_log2)
+                          : make_float2(0.f, 0.f);
+        }
     }
+    const bool single = p.Tnew == 1;  // every key below kv_end is visible
     int64_t row_lim[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) row_lim[r] = (r < p.Rv) ? p.start_pos + (r % p.Tnew) : -1;
 
-    float2 o2[R][E / 2];
+    float2 o2[R][EC / 2];
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
-        for (int j = 0; j < E / 2; ++j) o2[r][j] = make_float2(0.f, 0.f);
+        for (int j = 0; j < EC / 2; ++j) o2[r][j] = make_float2(0.f, 0.f);
     const int rb = lane / LPR;
     float m_run = -INFINITY, l_part = 0.f;
     float* scw = sc + warp * KW * R;
@@ -591,16 +624,23 @@ decode_wide_kernel(const DecodeParams p) {
         for (int gi = 0; gi < GPW; ++gi) {
             const int kw = gi * KPG + kslot;
             const int ki = warp * KW + kw;
-            float f[E];
-            load_piece<T, E>(kst + size_t(ki) * D + e0, f);
             float acc[R];
+            float2 a2[R];
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                float2 a2 = __fmul2_rn(q2[r][0], make_float2(f[0], f[1]));
+            for (int c = 0; c < NPC; ++c) {
+                float f[PE];
+                load_elems<T, PE>(kst + size_t(ki) * D + (c * LPK + sub) * PE, f);
 #pragma unroll
-                for (int j = 1; j < E / 2; ++j) a2 = __ffma2_rn(q2[r][j], make_float2(f[2 * j], f[2 * j + 1]), a2);
-                acc[r] = a2.x + a2.y;
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int j = 0; j < PE / 2; ++j) {
+                        const float2 kv = make_float2(f[2 * j], f[2 * j + 1]);
+                        if (c == 0 && j == 0) a2[r] = __fmul2_rn(q2[r][0], kv);
+                        else a2[r] = __ffma2_rn(q2[r][c * (PE / 2) + j], kv, a2[r]);
+                    }
             }
+#pragma unroll
+            for (int r = 0; r < R; ++r) acc[r] = a2[r].x + a2[r].y;
             int n = R;
 #pragma unroll
             for (int o = LPK / 2; o >= 1; o >>= 1) {
@@ -619,11 +659,13 @@ decode_wide_kernel(const DecodeParams p) {
                     acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
                 }
             }
-            const int64_t j = k0 + ki;
             bool vis = ki < nvalid;
+            if (!single) {
+                const int64_t j = k0 + ki;
 #pragma unroll
-            for (int r = 0; r < R; ++r)
-                if (r == my_row) vis = vis && (j <= row_lim[r]);
+                for (int r = 0; r < R; ++r)
+                    if (r == my_row) vis = vis && (j <= row_lim[r]);
+            }
             if (sub % (LPK / R) == 0) scw[kw * R + my_row] = vis ? acc[0] : -INFINITY;
         }
         __syncwarp();
@@ -660,7 +702,7 @@ decode_wide_kernel(const DecodeParams p) {
         }
         __syncwarp();
 
-        // C. rescale and accumulate P V
+        // C. rescale and accumulate P V: lanes split d, each walks the warp's keys
         {
             float a[R];
             bool any = false;
@@ -673,22 +715,21 @@ decode_wide_kernel(const DecodeParams p) {
 #pragma unroll
                 for (int r = 0; r < R; ++r)
 #pragma unroll
-                    for (int jj = 0; jj < E / 2; ++jj) o2[r][jj] = __fmul2_rn(o2[r][jj], make_float2(a[r], a[r]));
+                    for (int jj = 0; jj < EC / 2; ++jj) o2[r][jj] = __fmul2_rn(o2[r][jj], make_float2(a[r], a[r]));
             }
+            const int kv_here = min(KW, nvalid - warp * KW);
 #pragma unroll
-            for (int gi = 0; gi < GPW; ++gi) {
-                const int kw = gi * KPG + kslot;
-                const int ki = warp * KW + kw;
-                if (ki < nvalid) {
+            for (int kw = 0; kw < KW; ++kw) {
+                if (kw < kv_here) {
                     float pr[R];
 #pragma unroll
                     for (int r = 0; r < R; ++r) pr[r] = scw[kw * R + r];
-                    float f[E];
-                    load_piece<T, E>(vst + size_t(ki) * D + e0, f);
+                    float f[EC];
+                    load_elems<T, EC>(vst + size_t(warp * KW + kw) * D + lane * EC, f);
 #pragma unroll
                     for (int r = 0; r < R; ++r)
 #pragma unroll
-                        for (int jj = 0; jj < E / 2; ++jj)
+                        for (int jj = 0; jj < EC / 2; ++jj)
                             o2[r][jj] = __ffma2_rn(make_float2(pr[r], pr[r]),
                                                    make_float2(f[2 * jj], f[2 * jj + 1]), o2[r][jj]);
                 }
@@ -698,16 +739,7 @@ decode_wide_kernel(const DecodeParams p) {
         if (lane == 0) mbar_arrive(smem_u32(&bars[NST + st]));
     }
 
-    // ---- merge: key slots of a warp, then the warps of the CTA
-#pragma unroll
-    for (int o = LPK; o < 32; o <<= 1)
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int jj = 0; jj < E / 2; ++jj) {
-                o2[r][jj].x += __shfl_xor_sync(0xffffffffu, o2[r][jj].x, o);
-                o2[r][jj].y += __shfl_xor_sync(0xffffffffu, o2[r][jj].y, o);
-            }
+    // ---- merge the warps of the CTA
 #pragma unroll
     for (int o = LPR / 2; o >= 1; o >>= 1) l_part += __shfl_xor_sync(0xffffffffu, l_part, o);
 
@@ -719,15 +751,13 @@ decode_wide_kernel(const DecodeParams p) {
         mo[warp * R + rb] = m_run;
         lo[warp * R + rb] = l_part;
     }
-    if (kslot == 0) {
 #pragma unroll
-        for (int r = 0; r < R; ++r)
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int jj = 0; jj < E / 2; ++jj) {
-                oo[(warp * R + r) * D + e0 + 2 * jj] = o2[r][jj].x;
-                oo[(warp * R + r) * D + e0 + 2 * jj + 1] = o2[r][jj].y;
-            }
-    }
+        for (int jj = 0; jj < EC / 2; ++jj) {
+            oo[(warp * R + r) * D + lane * EC + 2 * jj] = o2[r][jj].x;
+            oo[(warp * R + r) * D + lane * EC + 2 * jj + 1] = o2[r][jj].y;
+        }
     asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
 
     const bool aborted = *abort_flag != 0;
