@@ -1,0 +1,60 @@
+"""Device-side failure detection without a GPU fault (needs a B200).
+
+Every wait inside the kernels is bounded.  The test hook makes the K/V
+producers issue no copies, so the consumers' waits run out after a short
+limit: the kernels must record ATTN_ERR_DEVICE_TIMEOUT, exit cleanly (TMEM
+freed, no copy left in flight) and leave the context usable, which the normal
+calls afterwards check against the oracle.  No fault, trap or hang is
+provoked: nothing waits without a bound.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import transformer_attention_causal_b200 as attn
+from oracle import attention as oracle
+from transformer_attention_causal_b200 import _lib, inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from transformer_attention_causal_b200.build import build
+
+    build()
+
+
+def test_bounded_waits_report_a_timeout_and_leave_the_context_usable():
+    lib = _lib.load()
+    scale = 1 / math.sqrt(128)
+    pq, pk, pv = inputs.qkv(1, 4, 2, 256, 256, 128, torch.bfloat16, seed=31)
+    dq, dk, dv = inputs.qkv(2, 8, 2, 1, 1000, 128, torch.bfloat16, seed=32)
+    assert attn.prefill_plan(torch.bfloat16, 1, 4, 2, 256, 128) == "tcgen05"
+    assert attn.cached_plan(torch.bfloat16, 2, 8, 2, 1, 1000, 1000, 128, 999) == "splitkv"
+    pq, pk, pv, dq, dk, dv = (t.cuda() for t in (pq, pk, pv, dq, dk, dv))
+    assert attn.device_status(reset=True) == _lib.OK
+    try:
+        attn.set_wait_timeout_ns(20_000_000)  # 20 ms
+        lib.attn_test_set_flags(1)
+        attn.prefill(pq, pk, pv, scale=scale)
+        assert attn.device_status(reset=True) == _lib.ERR_DEVICE_TIMEOUT
+        attn.cached(dq, dk, dv, start_pos=999, scale=scale)
+        assert attn.device_status(reset=True) == _lib.ERR_DEVICE_TIMEOUT
+    finally:
+        lib.attn_test_set_flags(0)
+        attn.set_wait_timeout_ns(0)
+    # the context is intact: normal calls run and match the oracle
+    out = attn.prefill(pq, pk, pv, scale=scale).float().cpu().numpy()
+    ref = oracle(pq.cpu(), pk.cpu(), pv.cpu(), scale=scale, causal=True)
+    err = np.abs(out - ref)
+    assert err.max() <= 1.5e-2 and err.mean() <= 2e-3
+    out = attn.cached(dq, dk, dv, start_pos=999, scale=scale).float().cpu().numpy()
+    ref = oracle(dq.cpu(), dk.cpu(), dv.cpu(), scale=scale, causal=True, start_pos=999)
+    err = np.abs(out - ref)
+    assert err.max() <= 1.5e-2 and err.mean() <= 2e-3
+    assert attn.device_status() == _lib.OK

@@ -24,7 +24,7 @@ KERNEL_NAMES = {KERNEL_NONE: "none", KERNEL_SIMT: "simt", KERNEL_TCGEN05: "tcgen
 
 EXPORTS = ("attn_prefill", "attn_cached", "attn_cached_workspace_size", "attn_prefill_plan",
            "attn_cached_plan", "attn_status_string", "attn_device_status",
-           "attn_set_wait_timeout_ns", "attn_version")
+           "attn_set_wait_timeout_ns", "attn_test_set_flags", "attn_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -64,6 +64,8 @@ def load() -> ctypes.CDLL:
             lib.attn_device_status.argtypes = [vp, c_int]
             lib.attn_set_wait_timeout_ns.restype = None
             lib.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+            lib.attn_test_set_flags.restype = None
+            lib.attn_test_set_flags.argtypes = [ctypes.c_uint32]
             lib.attn_version.restype = c_int
             lib.attn_version.argtypes = []
             _lib = lib

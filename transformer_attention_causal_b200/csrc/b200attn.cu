@@ -22,6 +22,7 @@ namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<uint32_t> g_test_flags{0};
 
 // Planning constants for B200: 148 SMs.  The wide decode kernel runs one
 // 512-thread CTA per SM with 120-key stages; the compact one (large row
@@ -299,6 +300,7 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
     dp.kv_end = pl.kv_end; dp.chunk = pl.chunk; dp.nsplit = pl.nsplit;
     dp.scale_log2 = scale * 1.4426950408889634f;
     dp.timeout_ns = g_timeout_ns.load();
+    dp.test_flags = g_test_flags.load();
     switch (pb.d) {
     case 64: return launch_decode_D<T, 64>(pl.R, pl.wide, dp, stream);
     case 128: return launch_decode_D<T, 128>(pl.R, pl.wide, dp, stream);
@@ -325,6 +327,7 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
     pp.units_per_level = pl.units_per_level;
     pp.scale_log2 = scale * 1.4426950408889634f;
     pp.timeout_ns = g_timeout_ns.load();
+    pp.test_flags = g_test_flags.load();
     constexpr size_t smem = prefill_smem_bytes<DCH>();
     auto kern = prefill_tcgen05_kernel<T, DCH>;
     static std::once_flag once[8];
@@ -467,6 +470,8 @@ attn_status_t attn_device_status(void* stream, int reset) {
 }
 
 void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs); }
+
+void attn_test_set_flags(uint32_t flags) { g_test_flags.store(flags); }
 
 int attn_version(void) { return 100; }
 

@@ -46,6 +46,7 @@ struct DecodeParams {
     int nsplit;
     float scale_log2;    // scale * log2(e)
     uint64_t timeout_ns;
+    uint32_t test_flags;  // kTestSkipLoads: issue no K/V copies (timeout-path tests)
 };
 
 template <int D, int R>
@@ -116,7 +117,8 @@ decode_splitkv_kernel(const DecodeParams p) {
         // ------------------------------------------------ producer
         if (lane == 0) {
             int issued = 0;
-            for (int it = 0; it < nstages; ++it) {
+            const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : nstages;
+            for (int it = 0; it < n_loads; ++it) {
                 const int st = it % NST;
                 const uint32_t ph = (it / NST) & 1;
                 if (!mbar_wait(smem_u32(&bars[NST + st]), ph ^ 1, p.timeout_ns, abort_flag)) break;
@@ -550,7 +552,8 @@ decode_wide_kernel(const DecodeParams p) {
     if (warp == NW) {
         if (lane == 0) {
             int issued = 0;
-            for (int it = 0; it < nstages; ++it) {
+            const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : nstages;
+            for (int it = 0; it < n_loads; ++it) {
                 const int st = it % NST;
                 if (!mbar_wait(smem_u32(&bars[NST + st]), ((it / NST) & 1) ^ 1, p.timeout_ns, abort_flag))
                     break;

@@ -52,6 +52,7 @@ struct PrefillParams {
     int units_per_level;
     float scale_log2;    // scale * log2(e)
     uint64_t timeout_ns;
+    uint32_t test_flags;  // kTestSkipLoads: issue no K/V copies (timeout-path tests)
 };
 
 constexpr int kPfThreads = 384;  // 12 warps
@@ -264,7 +265,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             const int zkv = b * p.Hkv + kvh;
             int issued = 0;
-            for (int i = 0; i < 2 * nmax; ++i) {
+            const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * nmax;
+            for (int i = 0; i < n_loads; ++i) {
                 const int st = i % NST;
                 if (!mbar_wait(smem_u32(&kv_empty[st]), ((i / NST) & 1) ^ 1, p.timeout_ns, abort_flag))
                     break;

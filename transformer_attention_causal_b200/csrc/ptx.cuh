@@ -16,6 +16,10 @@ __device__ unsigned int g_device_status;
 
 constexpr unsigned kStatusTimeout = 5u;  // == ATTN_ERR_DEVICE_TIMEOUT
 
+// Test hook (attn_test_set_flags): producers issue no K/V copies, so every
+// consumer's bounded wait runs out and the timeout path is exercised.
+constexpr uint32_t kTestSkipLoads = 1u;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
