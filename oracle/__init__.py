@@ -4,6 +4,6 @@ TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package; the product path (the
 CUDA library and its binding) never does.  It shares no code with the CUDA path.
 """
-from .attention import attention, build, library_path, num_cores, widen_bits
+from .attention import attention, build, library_path, num_cores, rope_append, widen_bits
 
-__all__ = ["attention", "build", "library_path", "num_cores", "widen_bits"]
+__all__ = ["attention", "build", "library_path", "num_cores", "rope_append", "widen_bits"]

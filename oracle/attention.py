@@ -56,6 +56,8 @@ def _bind(path: str):
     lib.oracle_widen_f16.restype = dbl
     lib.oracle_widen_f16.argtypes = [ctypes.c_uint16]
     lib.oracle_num_cores.restype = ctypes.c_int
+    lib.oracle_rope_append.restype = ctypes.c_int
+    lib.oracle_rope_append.argtypes = [vp, vp, ctypes.c_int, i64, i64, i64, i64, i64, dbl, vp, vp]
     return lib
 
 
@@ -174,4 +176,25 @@ def load_variant(path: str):
     return types.SimpleNamespace(
         attention=lambda *a, **kw: attention(*a, _lib_handle=handle, **kw),
         widen_bits=lambda *a, **kw: widen_bits(*a, _lib_handle=handle, **kw),
+        rope_append=lambda *a, **kw: rope_append(*a, _lib_handle=handle, **kw),
     )
+
+
+def rope_append(k_new, v_new, *, start_pos: int, base: float, _lib_handle=None):
+    """fp64 rows that a KV-cache append writes: K rotated with NeoX RoPE at
+    positions start_pos + t (base <= 0: no rotation), V unchanged.
+    k_new, v_new: [B, Hkv, Tnew, d].  Returns (k_rows, v_rows) float64."""
+    ka, code = _as_raw(k_new)
+    va, vcode = _as_raw(v_new)
+    if code != vcode or ka.shape != va.shape or ka.ndim != 4:
+        raise ValueError("k_new and v_new must be [B, Hkv, Tnew, d] of one dtype")
+    B, Hkv, Tnew, d = ka.shape
+    k_out = np.zeros(ka.shape, dtype=np.float64)
+    v_out = np.zeros(ka.shape, dtype=np.float64)
+    lib = _lib() if _lib_handle is None else _lib_handle
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    rc = lib.oracle_rope_append(ptr(ka), ptr(va), code, B, Hkv, Tnew, d, int(start_pos),
+                                float(base), ptr(k_out), ptr(v_out))
+    if rc != 0:
+        raise ValueError(f"oracle_rope_append rejected its arguments (code {rc})")
+    return k_out, v_out

@@ -223,3 +223,52 @@ int oracle_attention(const void* q, const void* k, const void* v, int dtype,
 }
 
 int oracle_num_cores(void) { return (int)sysconf(_SC_NPROCESSORS_ONLN); }
+
+/*
+ * KV-cache append with rotary position embedding on K (NeoX pairing).
+ *
+ * Follows "Hesper.Layers.Attention", fusedRopeKAndCacheWriteKernel (RoPE on
+ * the new K, written together with V into the cache slot at the token's
+ * position; the rotation partner of dimension i < d/2 is i + d/2) and
+ * kvWriteBatchKernelF16 (the same write without rotation), and "Grouped-Query
+ * Attention" §5.1 (apply_rope with offset = start_pos before the cache
+ * append).  The frequency of pair i is base^(-2i/d) — the pages leave that
+ * formula unrendered; this is the reading stated in the design notes.
+ *
+ * For every b < B, kv head h < Hkv, new token t < Tnew at position
+ * p = start_pos + t, and i < d/2 with a = p * base^(-2i/d):
+ *   K_out[i]       = K[i] cos a - K[i + d/2] sin a
+ *   K_out[i + d/2] = K[i + d/2] cos a + K[i] sin a
+ *   V_out          = V
+ * base <= 0 means no rotation.  Inputs k_new, v_new: [B, Hkv, Tnew, d];
+ * outputs (fp64) k_out, v_out: [B, Hkv, Tnew, d] (the rows to be written at
+ * positions start_pos .. start_pos + Tnew - 1).
+ */
+int oracle_rope_append(const void* k_new, const void* v_new, int dtype, int64_t B, int64_t Hkv,
+                       int64_t Tnew, int64_t d, int64_t start_pos, double base, double* k_out,
+                       double* v_out) {
+    if (B < 0 || Hkv < 0 || Tnew < 0 || d <= 0 || (d & 1) || start_pos < 0 || dtype < 0 ||
+        dtype > 3)
+        return -1;
+    const int64_t h = d / 2;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t kv = 0; kv < Hkv; ++kv)
+            for (int64_t t = 0; t < Tnew; ++t) {
+                const int64_t row = ((b * Hkv + kv) * Tnew + t) * d;
+                const double pos = (double)(start_pos + t);
+                for (int64_t i = 0; i < d; ++i) v_out[row + i] = load_elem(v_new, dtype, row + i);
+                for (int64_t i = 0; i < h; ++i) {
+                    const double x0 = load_elem(k_new, dtype, row + i);
+                    const double x1 = load_elem(k_new, dtype, row + i + h);
+                    if (base <= 0.0) {
+                        k_out[row + i] = x0;
+                        k_out[row + i + h] = x1;
+                        continue;
+                    }
+                    const double a = pos * pow(base, -2.0 * (double)i / (double)d);
+                    k_out[row + i] = x0 * cos(a) - x1 * sin(a);
+                    k_out[row + i + h] = x1 * cos(a) + x0 * sin(a);
+                }
+            }
+    return 0;
+}

@@ -2,7 +2,8 @@
 
 Each case compiles a copy of ``oracle/attn_oracle.c`` with one deliberate
 mistake planted in it (on the CPU, into a temporary directory) and runs every
-pin of ``test_oracle_pins.py`` against that copy: at least one pin must fail.
+pin of ``test_oracle_pins.py`` and ``test_oracle_rope_pins.py`` against that
+copy: at least one pin must fail.
 The unmodified oracle passes all of them (that file's own run).
 """
 import inspect
@@ -12,6 +13,7 @@ import subprocess
 import pytest
 
 import test_oracle_pins as pins
+import test_oracle_rope_pins as rope_pins
 from oracle.attention import load_variant
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle",
@@ -37,13 +39,25 @@ MUTANTS = [
     ("f16 subnormals scaled wrongly", [("ldexp((double)frac, -24)", "ldexp((double)frac, -25)")]),
     ("batch stride ignored for K/V", [("int64_t kv_base = (b * J->Hkv + kvh) * J->S_cap;",
                                        "int64_t kv_base = kvh * J->S_cap;")]),
+    ("RoPE partner adjacent", [("load_elem(k_new, dtype, row + i + h);",
+                                "load_elem(k_new, dtype, row + (i ^ 1));")]),
+    ("RoPE rotation reversed", [("k_out[row + i] = x0 * cos(a) - x1 * sin(a);",
+                                 "k_out[row + i] = x0 * cos(a) + x1 * sin(a);"),
+                                ("k_out[row + i + h] = x1 * cos(a) + x0 * sin(a);",
+                                 "k_out[row + i + h] = x1 * cos(a) - x0 * sin(a);")]),
+    ("RoPE frequency exponent halved", [("pow(base, -2.0 * (double)i / (double)d)",
+                                         "pow(base, -1.0 * (double)i / (double)d)")]),
+    ("RoPE position ignores start_pos", [("const double pos = (double)(start_pos + t);",
+                                          "const double pos = (double)t;")]),
 ]
 
 
 def _pin_calls(golden_dir):
-    """Every test function of the pin module, with its parameter sets."""
+    """Every test function of the pin modules, with its parameter sets."""
     calls = []
-    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+    members = inspect.getmembers(pins, inspect.isfunction) + \
+        inspect.getmembers(rope_pins, inspect.isfunction)
+    for name, fn in members:
         if not name.startswith("test_"):
             continue
         marks = getattr(fn, "pytestmark", [])
@@ -76,6 +90,7 @@ def test_planted_mistake_fails_a_pin(name, edits, tmp_path, golden_dir, monkeypa
     variant = load_variant(str(lib))
     monkeypatch.setattr(pins, "attention", variant.attention)
     monkeypatch.setattr(pins, "widen_bits", variant.widen_bits)
+    monkeypatch.setattr(rope_pins, "rope_append", variant.rope_append)
     failed = []
     for test_name, fn, kwargs in _pin_calls(golden_dir):
         try:
