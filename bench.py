@@ -6,7 +6,9 @@
 One step = one call of the library on one batch of the workload (default: the
 BitNet-3B-shaped causal MHA prefill, B=1, H=32, T=2048, d=80, bf16).  The
 line also carries the cached-decode half of the metric (GQA decode, B=64,
-H=32/8, S=8192, d=128, bf16) measured the same way, with its own roofline.
+H=32/8, S=8192, d=128, bf16) and the KV-cache append with RoPE on K of the
+GQA prefill's keys and values (B=8, Hkv=8, 4096 tokens, d=128, bf16), each
+measured the same way with its own roofline.
 
 Timing: W untimed steps, then exactly K timed steps bracketed by a barrier and
 torch.cuda.synchronize() on both sides.  Before every timed call L2 is flushed
@@ -50,12 +52,17 @@ WORKLOADS = {
                             S=8192, d=128),
     "mqa_chunked_prefill_f16": dict(kind="cached", dtype="f16", B=32, H=8, Hkv=1, Tnew=512,
                                     start=3584, S=4096, d=128),
+    # the step before attention: the GQA prefill's 4096 new keys (RoPE) and values
+    # written into an empty cache
+    "kv_append_rope_gqa16x8_bf16": dict(kind="append", dtype="bf16", B=8, H=16, Hkv=8,
+                                        Tnew=4096, start=0, S=4096, d=128, base=10000.0),
 }
 DEFAULT_WORKLOAD = "bitnet3b_mha_prefill_bf16"
 DECODE_WORKLOAD = "gqa_decode_bf16"
+APPEND_WORKLOAD = "kv_append_rope_gqa16x8_bf16"
 TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
 KERNEL_SOURCES = {"tcgen05": "prefill_tcgen05.cuh", "splitkv": "decode_splitkv.cuh",
-                  "simt": "simt_attn.cuh"}
+                  "simt": "simt_attn.cuh", "append": "kv_append.cuh"}
 
 
 # ------------------------------------------------------------------ workload algebra
@@ -84,15 +91,24 @@ def algorithmic_flops(w):
     return 4 * w["d"] * w["B"] * w["H"] * visible_pairs(w)
 
 
+def esize(w):
+    return 2 if w["dtype"] in ("bf16", "f16") else 4
+
+
 def algorithmic_bytes(w):
-    """Q read + the visible K/V rows read once per K/V head + O written."""
-    esz = 2 if w["dtype"] in ("bf16", "f16") else 4
+    """Attention: Q read + the visible K/V rows read once per K/V head + O
+    written.  Append: the new K and V rows read once and written once."""
+    esz = esize(w)
+    if w["kind"] == "append":
+        return 4 * w["B"] * w["Hkv"] * w["Tnew"] * w["d"] * esz
     kv_vis = min(kv_len(w), start_pos(w) + q_len(w))
     q_o = 2 * w["B"] * w["H"] * q_len(w) * w["d"] * esz
     return q_o + 2 * w["B"] * w["Hkv"] * kv_vis * w["d"] * esz
 
 
 def bound(w):
+    if w["kind"] == "append":
+        return "hbm"
     return "hbm" if w["kind"] == "cached" and q_len(w) * w["H"] // w["Hkv"] <= 16 else "tensor"
 
 
@@ -101,6 +117,10 @@ def config_of(name, w, world):
            "dtype": w["dtype"], "causal": True, "scale": f"1/sqrt({w['d']})"}
     if w["kind"] == "prefill":
         cfg["T"] = w["T"]
+    elif w["kind"] == "append":
+        cfg = {"workload": name, "B": w["B"], "Hkv": w["Hkv"], "d": w["d"], "dtype": w["dtype"],
+               "Tnew": w["Tnew"], "start_pos": w["start"], "S_cap": w["S"],
+               "rope": f"NeoX, base {w['base']:g}"}
     else:
         cfg.update(Tnew=w["Tnew"], start_pos=w["start"], S=w["S"])
     cfg["l2"] = "flushed by a 256 MiB write before every timed call"
@@ -231,11 +251,23 @@ class Case:
         dt = TORCH_DTYPE[w["dtype"]]
         self.dtype = dt
         Tq, S = q_len(w), kv_len(w)
+        if w["kind"] == "append":
+            k_new = inputs.normal((w["B"], w["Hkv"], Tq, w["d"]), seed, 1, dt)
+            v_new = inputs.normal((w["B"], w["Hkv"], Tq, w["d"]), seed, 2, dt)
+            self.host = [t.pin_memory() for t in (k_new, v_new)]
+            self.dev_in = [t.to(device, non_blocking=True) for t in self.host]
+            self.dev_out = [torch.zeros((w["B"], w["Hkv"], S, w["d"]), dtype=dt, device=device)
+                            for _ in range(2)]
+            self.host_out = [torch.empty(t.shape, dtype=dt).pin_memory() for t in self.dev_out]
+            self.kernel, self.launches, self.device = "append", 1, device
+            return
         q, k, v = inputs.qkv(w["B"], w["H"], w["Hkv"], Tq, S, w["d"], dt, seed=seed)
         self.host = [t.pin_memory() for t in (q, k, v)]
         self.q, self.k, self.v = (t.to(device, non_blocking=True) for t in self.host)
         self.out = torch.empty_like(self.q)
-        self.out_host = torch.empty(self.out.shape, dtype=dt).pin_memory()
+        self.dev_in, self.dev_out = [self.q, self.k, self.v], [self.out]
+        self.host_out = [torch.empty(self.out.shape, dtype=dt).pin_memory()]
+        self.device = device
         self.scale = 1.0 / math.sqrt(w["d"])
         if w["kind"] == "prefill":
             self.kernel = attn.prefill_plan(dt, w["B"], w["H"], w["Hkv"], Tq, w["d"])
@@ -253,7 +285,10 @@ class Case:
 
     def call(self):
         w = self.w
-        if w["kind"] == "prefill":
+        if w["kind"] == "append":
+            self.attn.kv_append_rope(*self.dev_in, *self.dev_out, start_pos=w["start"],
+                                     rope_base=w["base"])
+        elif w["kind"] == "prefill":
             self.attn.prefill(self.q, self.k, self.v, scale=self.scale, causal=True, out=self.out)
         else:
             self.attn.cached(self.q, self.k, self.v, start_pos=w["start"], scale=self.scale,
@@ -263,7 +298,7 @@ class Case:
 def time_device(case, steps, warmup, dist_ctx):
     """Mean per-call device time (ms) over `steps` timed calls, L2 flushed
     before each; returns (kernel_ms, bracket_ms)."""
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=case.q.device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=case.device)
     for _ in range(warmup):
         flush.zero_()
         case.call()
@@ -290,11 +325,11 @@ def time_e2e(case, steps, warmup, dist_ctx):
     """Per-step time (ms) with the inputs copied host -> device from pinned
     memory and the output copied back, every step."""
     def step():
-        case.q.copy_(case.host[0], non_blocking=True)
-        case.k.copy_(case.host[1], non_blocking=True)
-        case.v.copy_(case.host[2], non_blocking=True)
+        for dev, host in zip(case.dev_in, case.host):
+            dev.copy_(host, non_blocking=True)
         case.call()
-        case.out_host.copy_(case.out, non_blocking=True)
+        for host, dev in zip(case.host_out, case.dev_out):
+            host.copy_(dev, non_blocking=True)
 
     for _ in range(warmup):
         step()
@@ -309,7 +344,7 @@ def time_e2e(case, steps, warmup, dist_ctx):
     torch.cuda.synchronize()
     dist_ctx.barrier()
     h2d = sum(t.numel() * t.element_size() for t in case.host)
-    d2h = case.out_host.numel() * case.out_host.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in case.host_out)
     return b0.elapsed_time(b1) / steps, h2d, d2h
 
 
@@ -369,46 +404,84 @@ def roofline(w, kernel_ms, kernel, name, peaks, peak_src):
             "kernel": kernel}
 
 
+class OracleSample:
+    """The fp64 oracle, as it stands, on seeded random samples of a workload:
+    query rows for attention, (batch, token) rows for the append.  Work is
+    counted in the workload's own unit: the FLOPs of the sampled rows, or
+    their share of the algorithmic bytes."""
+
+    def __init__(self, w, seed=0):
+        from transformer_attention_causal_b200 import inputs
+
+        self.w = w
+        dt = TORCH_DTYPE[w["dtype"]]
+        self.unit = "GB/s" if bound(w) == "hbm" else "TFLOP/s"
+        if w["kind"] == "append":
+            shape = (w["B"], w["Hkv"], w["Tnew"], w["d"])
+            self.k_new = inputs.normal(shape, seed, 1, dt)
+            self.v_new = inputs.normal(shape, seed, 2, dt)
+            self.total = w["B"] * w["Tnew"]
+            self.what = "(batch, token) rows of"
+        else:
+            self.q, self.k, self.v = inputs.qkv(w["B"], w["H"], w["Hkv"], q_len(w), kv_len(w),
+                                                w["d"], dt, seed=seed)
+            self.total = w["B"] * w["H"] * q_len(w)
+            self.what = "query rows of"
+        whole = algorithmic_bytes(w) / 1e9 if self.unit == "GB/s" else algorithmic_flops(w) / 1e12
+        self.per_unit = whole / self.total
+
+    def run(self, n, rng):
+        """Oracle time (s), work and count of one sample of n rows."""
+        import numpy as np
+
+        from oracle import attention as oracle_attention
+        from oracle import rope_append
+
+        w = self.w
+        n = int(min(n, self.total))
+        if w["kind"] == "append":
+            T = w["Tnew"]
+            jobs, left = [], n
+            while left > 0:
+                m = min(left, T)
+                b, t0 = int(rng.integers(w["B"])), int(rng.integers(T - m + 1))
+                jobs.append((self.k_new[b:b + 1, :, t0:t0 + m].contiguous(),
+                             self.v_new[b:b + 1, :, t0:t0 + m].contiguous(), w["start"] + t0))
+                left -= m
+            t0 = time.perf_counter()
+            for kn, vn, pos in jobs:
+                rope_append(kn, vn, start_pos=pos, base=w["base"])
+            return time.perf_counter() - t0, n * self.per_unit, n
+        rows = np.sort(rng.choice(self.total, size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle_attention(self.q, self.k, self.v, scale=1 / math.sqrt(w["d"]), causal=True,
+                         start_pos=start_pos(w), rows=rows)
+        secs = time.perf_counter() - t0
+        if self.unit == "GB/s":
+            return secs, n * self.per_unit, n
+        i = rows % q_len(w)
+        return secs, float(np.sum(4 * w["d"] * (start_pos(w) + i + 1))) / 1e12, n
+
+    def sized(self, target_s, rng):
+        """Rows that take the oracle about target_s seconds, from a pilot run."""
+        from oracle import num_cores
+
+        secs, work, _ = self.run(4 * num_cores(), rng)
+        return int(min(self.total, max(16, target_s * (work / max(secs, 1e-6)) / self.per_unit)))
+
+
 def cpu_baseline(w, name, target_s=10.0):
-    """The fp64 oracle, as it stands, on a bounded seeded row sample of the
-    workload, on every host core."""
+    """The oracle on a bounded sample of the workload, on every host core."""
     import numpy as np
 
-    from oracle import attention as oracle_attention
     from oracle import num_cores
-    from transformer_attention_causal_b200 import inputs
 
-    dt = TORCH_DTYPE[w["dtype"]]
-    Tq, S, s0 = q_len(w), kv_len(w), start_pos(w)
-    q, k, v = inputs.qkv(w["B"], w["H"], w["Hkv"], Tq, S, w["d"], dt, seed=0)
-    total_rows = w["B"] * w["H"] * Tq
     rng = np.random.default_rng(0)
-
-    def row_flops(rows):
-        i = np.asarray(rows) % Tq
-        return float(np.sum(4 * w["d"] * (s0 + i + 1)))
-
-    def run(n):
-        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
-        t0 = time.perf_counter()
-        oracle_attention(q, k, v, scale=1 / math.sqrt(w["d"]), causal=True, start_pos=s0,
-                         rows=rows)
-        return time.perf_counter() - t0, row_flops(rows), len(rows)
-
-    dt_pilot, fl_pilot, _ = run(4 * num_cores())
-    rate = fl_pilot / max(dt_pilot, 1e-6)
-    per_row = algorithmic_flops(w) / total_rows
-    n = int(min(total_rows, max(64, target_s * rate / per_row)))
-    secs, flops, nrows = run(n)
-    if bound(w) == "hbm":
-        esz = 2 if w["dtype"] != "f32" else 4
-        byts = nrows * (2 * w["d"] * esz + 2 * min(S, s0 + Tq) * w["d"] * esz)
-        value, unit = byts / secs / 1e9, "GB/s"
-    else:
-        value, unit = flops / secs / 1e12, "TFLOP/s"
-    return {"value": value, "unit": unit, "cores": num_cores(), "kind": "oracle",
-            "sample": f"{nrows} seeded random rows of {total_rows} ({secs:.1f} s, "
-                      f"fp64 two-pass softmax)"}
+    sample = OracleSample(w)
+    n = sample.sized(target_s, rng)
+    secs, work, nrows = sample.run(n, rng)
+    return {"value": work / secs, "unit": sample.unit, "cores": num_cores(), "kind": "oracle",
+            "sample": f"{nrows} seeded random {sample.what} {sample.total} ({secs:.1f} s, fp64)"}
 
 
 def whole_job_value(world: int, work_per_step: float, slowest_ms: float) -> float:
@@ -477,21 +550,25 @@ def run_ours(args, dist_ctx):
         "clocks": clocks,
         "device_status": status,
     }
-    if not args.no_decode and name != DECODE_WORKLOAD:
-        del case
+    legs = [] if args.no_decode else [("decode", DECODE_WORKLOAD), ("append", APPEND_WORKLOAD)]
+    del case
+    for key, leg in legs:
+        if leg == name:
+            continue
         torch.cuda.empty_cache()
-        wd = WORKLOADS[DECODE_WORKLOAD]
-        dcase = Case(DECODE_WORKLOAD, wd, device)
-        dsteps = max(args.steps, 5)
-        d_ms, _ = time_device(dcase, dsteps, max(args.warmup, 3), dist_ctx)
-        d_ms = dist_ctx.max(d_ms)
-        line["decode"] = {
-            "workload": DECODE_WORKLOAD,
-            "value": round(N * algorithmic_bytes(wd) / 1e9 / (d_ms * 1e-3), 2),
-            "unit": "GB/s", "ms_per_step": round(d_ms, 5), "steps": dsteps,
-            "gpu_launches": dsteps * dcase.launches,
-            "roofline": roofline(wd, d_ms, dcase.kernel, DECODE_WORKLOAD, peaks, peak_src),
+        wl = WORKLOADS[leg]
+        lcase = Case(leg, wl, device)
+        lsteps = max(args.steps, 5)
+        l_ms, _ = time_device(lcase, lsteps, max(args.warmup, 3), dist_ctx)
+        l_ms = dist_ctx.max(l_ms)
+        line[key] = {
+            "workload": leg,
+            "value": round(N * algorithmic_bytes(wl) / 1e9 / (l_ms * 1e-3), 2),
+            "unit": "GB/s", "ms_per_step": round(l_ms, 5), "steps": lsteps,
+            "gpu_launches": lsteps * lcase.launches,
+            "roofline": roofline(wl, l_ms, lcase.kernel, leg, peaks, peak_src),
         }
+        del lcase
     if dist_ctx.rank == 0 and N == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, name)
     if dist_ctx.rank == 0:
@@ -504,45 +581,22 @@ def run_reference(args, dist_ctx):
         return
     import numpy as np
 
-    from oracle import attention as oracle_attention
     from oracle import num_cores
-    from transformer_attention_causal_b200 import inputs
 
     name = args.workload
     w = workload(name, args.batch)
-    dt = TORCH_DTYPE[w["dtype"]]
-    Tq, S, s0 = q_len(w), kv_len(w), start_pos(w)
-    q, k, v = inputs.qkv(w["B"], w["H"], w["Hkv"], Tq, S, w["d"], dt, seed=0)
-    total_rows = w["B"] * w["H"] * Tq
     per_step_s = min(5.0, 150.0 / max(1, args.steps + args.warmup))
     rng = np.random.default_rng(1)
-    unit = "GB/s" if bound(w) == "hbm" else "TFLOP/s"
-    esz = 2 if w["dtype"] != "f32" else 4
-
-    def work_of(rows):
-        i = np.asarray(rows) % Tq
-        if unit == "GB/s":
-            return float(len(rows) * (2 * w["d"] * esz + 2 * min(S, s0 + Tq) * w["d"] * esz)) / 1e9
-        return float(np.sum(4 * w["d"] * (s0 + i + 1))) / 1e12
-
-    def step(n):
-        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
-        t0 = time.perf_counter()
-        oracle_attention(q, k, v, scale=1 / math.sqrt(w["d"]), causal=True, start_pos=s0,
-                         rows=rows)
-        return time.perf_counter() - t0, work_of(rows), len(rows)
-
-    secs, work, _ = step(4 * num_cores())
-    per_row = (algorithmic_flops(w) / 1e12 if unit == "TFLOP/s" else algorithmic_bytes(w) / 1e9) \
-        / total_rows
-    n = int(min(total_rows, max(16, per_step_s * (work / max(secs, 1e-6)) / per_row)))
+    sample = OracleSample(w)
+    n = sample.sized(per_step_s, rng)
     for _ in range(args.warmup):
-        step(n)
-    tot_s, tot_w, nrows = 0.0, 0.0, 0
+        sample.run(n, rng)
+    tot_s, tot_w = 0.0, 0.0
     for _ in range(args.steps):
-        s_, w_, r_ = step(n)
-        tot_s, tot_w, nrows = tot_s + s_, tot_w + w_, nrows + r_
+        s_, w_, _ = sample.run(n, rng)
+        tot_s, tot_w = tot_s + s_, tot_w + w_
     value = tot_w / tot_s
+    unit = sample.unit
     line = {
         "metric": METRIC, "impl": "reference", "value": value, "unit": unit, "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup,
@@ -551,7 +605,7 @@ def run_reference(args, dist_ctx):
         "data": "synthetic: i.i.d. N(0,1) from seed 0, rounded to the dtype",
         "config": config_of(name, w, 1),
         "cpu_baseline": {"value": value, "unit": unit, "cores": num_cores(), "kind": "oracle",
-                         "sample": f"{n} seeded random rows of {total_rows} per step"},
+                         "sample": f"{n} seeded random {sample.what} {sample.total} per step"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -564,7 +618,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode half")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode and append legs of the line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (smaller profiling captures)")

@@ -135,6 +135,32 @@ ATTN_API attn_status_t attn_cached_noalloc(const void* q, const void* k_hist, co
                                            int64_t S_cap, int64_t d, int64_t start_pos,
                                            float scale, void* stream);
 
+/*
+ * Append new tokens' keys and values to a KV cache, rotating the keys with
+ * rotary position embedding on the way ("Hesper.Layers.Attention", the fused
+ * RoPE-K and cache-write kernels and the no-RoPE batched write;
+ * "Grouped-Query Attention" §5.1, apply_rope at offset start_pos before the
+ * cache append).  For new token t at position p = start_pos + t and
+ * i < d/2, with angle a = p * rope_base^(-2i/d) (NeoX pairing: dimension i
+ * turns together with i + d/2):
+ *   K_cache[p][i]       = K[t][i] cos a - K[t][i + d/2] sin a
+ *   K_cache[p][i + d/2] = K[t][i + d/2] cos a + K[t][i] sin a
+ *   V_cache[p]          = V[t]
+ * rope_base <= 0 writes K unrotated.  The angle is reduced in double
+ * precision, then rotated in fp32; results are rounded to nearest-even.
+ *   k_new, v_new: [B, Hkv, Tnew, d]; k_cache, v_cache: [B, Hkv, S_cap, d];
+ *   rows start_pos .. start_pos + Tnew - 1 of every (b, kv head) are written,
+ *   nothing else is touched.
+ * Errors (nothing launched): ATTN_ERR_INVALID_ARG for a null or unaligned
+ * (16-byte) pointer, negative size, start_pos + Tnew > S_cap, non-finite
+ * rope_base, or d not a multiple of 8 (4 for ATTN_F32); ATTN_ERR_UNSUPPORTED
+ * for d > 256, Hkv > 65536 or B * Tnew > 2^31.  An empty append (B, Hkv or Tnew = 0) returns ATTN_OK.
+ */
+ATTN_API attn_status_t attn_kv_append_rope(const void* k_new, const void* v_new, void* k_cache,
+                                           void* v_cache, attn_dtype_t dtype, int64_t B,
+                                           int64_t Hkv, int64_t Tnew, int64_t S_cap, int64_t d,
+                                           int64_t start_pos, float rope_base, void* stream);
+
 /* Bytes of workspace attn_cached needs for this problem (0 if none).  Pure
  * host arithmetic; valid without a GPU.  Returns 0 for arguments that
  * attn_cached would reject. */

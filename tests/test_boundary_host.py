@@ -147,3 +147,28 @@ def test_workspace_size_is_zero_without_splits(lib):
     assert lib.attn_cached_workspace_size(BF16, 1, 4, 1, 1, 65536, 128, 65535) > 0
     # rejected arguments report 0
     assert lib.attn_cached_workspace_size(BF16, 1, 4, 3, 1, 64, 128, 63) == 0
+
+
+def append(lib, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, dt=BF16, B=1, Hkv=2, Tnew=4, S_cap=16, d=64,
+           start_pos=3, base=10000.0):
+    return lib.attn_kv_append_rope(k, v, kc, vc, dt, B, Hkv, Tnew, S_cap, d, start_pos, base, None)
+
+
+@pytest.mark.parametrize("kwargs", [
+    dict(k=None), dict(v=None), dict(kc=None), dict(vc=None),
+    dict(kc=MISALIGNED), dict(v=MISALIGNED),
+    dict(start_pos=13),                # 13 + 4 > 16
+    dict(start_pos=-1), dict(B=-1), dict(Tnew=-2), dict(S_cap=-1),
+    dict(d=0), dict(d=60), dict(d=6, dt=F32), dict(dt=5),
+    dict(base=float("nan")), dict(base=float("inf")),
+])
+def test_append_rejects_invalid_arguments(lib, kwargs):
+    assert append(lib, **kwargs) == INVALID
+
+
+def test_append_limits_and_empty_calls(lib):
+    assert append(lib, d=264) == UNSUPPORTED
+    assert append(lib, d=260, dt=F32) == UNSUPPORTED
+    # nothing to write: no launch, null pointers allowed
+    assert append(lib, k=None, v=None, kc=None, vc=None, Tnew=0) == 0
+    assert append(lib, k=None, v=None, kc=None, vc=None, B=0) == 0

@@ -16,8 +16,8 @@ import ctypes
 from . import _lib
 from ._lib import AttnError
 
-__all__ = ["prefill", "cached", "cached_workspace_size", "prefill_plan", "cached_plan",
-           "device_status", "set_wait_timeout_ns", "AttnError"]
+__all__ = ["prefill", "cached", "kv_append_rope", "cached_workspace_size", "prefill_plan",
+           "cached_plan", "device_status", "set_wait_timeout_ns", "AttnError"]
 
 
 def _torch():
@@ -110,6 +110,28 @@ def cached(q, k_hist, v_hist, *, start_pos: int, scale: float, S: int | None = N
     if st != _lib.OK:
         raise AttnError(st, "attn_cached")
     return out
+
+
+def kv_append_rope(k_new, v_new, k_cache, v_cache, *, start_pos: int, rope_base: float = 10000.0,
+                   stream=None):
+    """Write the new tokens' K (rotated with NeoX RoPE at positions
+    start_pos + t; rope_base <= 0: unrotated) and V into the caches.
+    k_new, v_new [B, Hkv, Tnew, d]; k_cache, v_cache [B, Hkv, S_cap, d]."""
+    _check(k_new, v_new, k_cache, v_cache)
+    B, Hkv, Tnew, d = k_new.shape
+    S_cap = k_cache.shape[2]
+    if tuple(v_new.shape) != tuple(k_new.shape) or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or tuple(k_cache.shape[:2]) != (B, Hkv) or k_cache.shape[3] != d:
+        raise ValueError("expected k_new, v_new [B, Hkv, Tnew, d] and caches [B, Hkv, S_cap, d]")
+    if not (k_new.dtype == v_new.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("all four tensors must share one dtype")
+    st = _lib.load().attn_kv_append_rope(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                         _dtype_code(k_new), B, Hkv, Tnew, S_cap, d,
+                                         int(start_pos), float(rope_base),
+                                         _stream_handle(stream, k_new.device))
+    if st != _lib.OK:
+        raise AttnError(st, "attn_kv_append_rope")
+    return k_cache, v_cache
 
 
 def prefill_plan(dtype, B, H, Hkv, T, d, causal=True) -> str:

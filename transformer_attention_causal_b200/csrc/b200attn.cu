@@ -13,6 +13,7 @@
 
 #include "b200attn.h"
 #include "decode_splitkv.cuh"
+#include "kv_append.cuh"
 #include "prefill_tcgen05.cuh"
 #include "simt_attn.cuh"
 
@@ -381,7 +382,67 @@ attn_status_t check_pointers(const Problem& pb, const void* q, const void* k, co
 
 }  // namespace
 
+namespace {
+
+template <typename T, int KB>
+attn_status_t run_append(const AppendParams& ap, int threads, cudaStream_t stream) {
+    const int64_t groups = (int64_t(ap.Tnew) + ap.tok_per_cta - 1) / ap.tok_per_cta;
+    const int64_t blocks = int64_t(ap.B) * groups;
+    if (blocks > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+    kv_append_rope_kernel<T, KB><<<unsigned(blocks), threads, 0, stream>>>(ap);
+    return launch_status();
+}
+
+template <typename T>
+attn_status_t launch_append(AppendParams& ap, cudaStream_t stream) {
+    const int esz = int(sizeof(T));
+    const int half_bytes = ap.d / 2 * esz;
+    const int kb = half_bytes % 16 == 0 ? 16 : 8;   // d/2 * esz is a multiple of 8
+    ap.half_units = half_bytes / kb;
+    const int per_tok = 2 * ap.Hkv * ap.half_units;
+    ap.div_tok = FastDiv(uint32_t(per_tok));
+    ap.div_row = FastDiv(uint32_t(ap.half_units));
+    const int threads = std::min(256, (per_tok + 31) / 32 * 32);
+    // as many tokens as fill every thread's units, at most kAppendMaxTok
+    ap.tok_per_cta = std::max(1, std::min(std::min(kAppendMaxTok, ap.Tnew),
+                                          threads * kAppendUnits / per_tok));
+    return kb == 16 ? run_append<T, 16>(ap, threads, stream) : run_append<T, 8>(ap, threads, stream);
+}
+
+}  // namespace
+
 extern "C" {
+
+attn_status_t attn_kv_append_rope(const void* k_new, const void* v_new, void* k_cache,
+                                  void* v_cache, attn_dtype_t dtype, int64_t B, int64_t Hkv,
+                                  int64_t Tnew, int64_t S_cap, int64_t d, int64_t start_pos,
+                                  float rope_base, void* stream) {
+    if (dtype != ATTN_F32 && dtype != ATTN_BF16 && dtype != ATTN_F16) return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || Hkv < 0 || Tnew < 0 || S_cap < 0 || d < 0 || start_pos < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(rope_base)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0 || Tnew == 0) return ATTN_OK;
+    const int64_t dmult = dtype == ATTN_F32 ? 4 : 8;
+    if (d == 0 || d % dmult != 0) return ATTN_ERR_INVALID_ARG;
+    if (d > kAppendMaxD) return ATTN_ERR_UNSUPPORTED;
+    if (start_pos + Tnew > S_cap) return ATTN_ERR_INVALID_ARG;
+    if (!k_new || !v_new || !k_cache || !v_cache) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+        return ATTN_ERR_INVALID_ARG;
+    if (B * Tnew > (int64_t(1) << 31) || Hkv > (int64_t(1) << 16)) return ATTN_ERR_UNSUPPORTED;
+    AppendParams ap{};
+    ap.k_new = k_new; ap.v_new = v_new; ap.k_cache = k_cache; ap.v_cache = v_cache;
+    ap.B = int(B); ap.Hkv = int(Hkv); ap.Tnew = int(Tnew); ap.d = int(d);
+    ap.S_cap = S_cap; ap.start_pos = start_pos;
+    ap.rotate = rope_base > 0.f ? 1 : 0;
+    // inverse frequencies base^(-2i/d), formed in double on the host
+    for (int64_t i = 0; ap.rotate && i < d / 2; ++i)
+        ap.inv_freq[i] = std::pow(double(rope_base), -2.0 * double(i) / double(d));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == ATTN_F32) return launch_append<float>(ap, s);
+    if (dtype == ATTN_BF16) return launch_append<__nv_bfloat16>(ap, s);
+    return launch_append<__half>(ap, s);
+}
 
 attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
                            attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t T,
