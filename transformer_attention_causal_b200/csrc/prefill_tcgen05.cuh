@@ -172,6 +172,40 @@ __device__ __forceinline__ SlotInfo prefill_slot(const PrefillParams& p, int h, 
     return s;
 }
 
+// S_s = Q_s K^T over d/16 k-steps.  Descriptors advance by adding (byte
+// offset >> 4) to their start-address field; the offsets are compile-time
+// constants, so each MMA issues without a descriptor being rebuilt (an MMA
+// stream whose descriptors are rebuilt per instruction issues more slowly than
+// the tensor pipe retires it).
+template <int DCH>
+__device__ __forceinline__ void issue_S(uint64_t dQ0, uint64_t dK0, uint32_t tmem, uint32_t idS,
+                                        int nk, int s, int st) {
+    constexpr uint32_t kStageStep = (DCH * kChunkBytes) >> 4;
+    const uint64_t a0 = dQ0 + uint64_t(uint32_t(s) * kStageStep);
+    const uint64_t b0 = dK0 + uint64_t(uint32_t(st) * kStageStep);
+    const uint32_t dS = tmem + s * 128;
+#pragma unroll
+    for (int kk = 0; kk < 4 * DCH; ++kk) {
+        if (kk >= nk) break;
+        const uint64_t off = uint64_t(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+        mma_ss(dS, a0 + off, b0 + off, idS, kk > 0 ? 1u : 0u);
+    }
+}
+
+// O_s (+)= P_s V for keys 16*K0 .. 16*K0 + 63 (P read from TMEM).
+template <int K0, int DCH>
+__device__ __forceinline__ void issue_PV(uint64_t dV0, uint32_t tmem, uint32_t idO, int s, int st,
+                                         bool accumulate) {
+    constexpr uint32_t kStageStep = (DCH * kChunkBytes) >> 4;
+    const uint64_t b0 = dV0 + uint64_t(uint32_t(st) * kStageStep);
+    const uint32_t dO = tmem + 256 + s * 128;
+    const uint32_t aP = tmem + s * 128;
+#pragma unroll
+    for (int kk = K0; kk < K0 + 4; ++kk)
+        mma_ts(dO, aP + kk * 8, b0 + uint64_t((kk * 2048) >> 4), idO,
+               (accumulate || kk > 0) ? 1u : 0u);
+}
+
 template <typename T, int DCH>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -290,23 +324,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             const uint32_t idS = idesc_f16(kBF16, 128, 128, false);
             const uint32_t idO = idesc_f16(kBF16, 128, p.d, true);
             const int nk = p.d / 16;
-            auto issue_S = [&](int s, int st) {
-                for (int kk = 0; kk < nk; ++kk) {
-                    const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-                    const uint64_t a = smem_desc_sw128(sQ + s * DCH * kChunkBytes + off, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(sRing + st * DCH * kChunkBytes + off, 16, 1024);
-                    mma_ss(tmem + s * 128, a, bd, idS, kk > 0 ? 1u : 0u);
-                }
-            };
-            auto issue_PV = [&](int s, int st, bool accumulate, int k0) {
-#pragma unroll
-                for (int kk = k0; kk < k0 + 4; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(sRing + st * DCH * kChunkBytes + kk * 2048,
-                                                        kChunkBytes, 1024);
-                    mma_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8, bd, idO,
-                           (accumulate || kk > 0) ? 1u : 0u);
-                }
-            };
+            const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t dK0 = smem_desc_sw128(sRing, 16, 1024);
+            const uint64_t dV0 = smem_desc_sw128(sRing, kChunkBytes, 1024);
             bool ok = true;
             for (int s = 0; s < 2 && ok; ++s)
                 if (slot[s].n_kv > 0) ok = mbar_wait(smem_u32(&q_full[s]), 0, p.timeout_ns, abort_flag);
@@ -315,7 +335,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tc_fence_after();
                 for (int s = 0; s < 2; ++s) {
                     if (slot[s].n_kv == 0) continue;
-                    issue_S(s, 0);
+                    issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, 0);
                     mma_commit(smem_u32(&s_full[s]));
                 }
                 mma_commit(smem_u32(&kv_empty[0]));
@@ -338,16 +358,16 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                         break;
                     }
                     tc_fence_after();
-                    issue_PV(s, stV, n > 0, 0);
+                    issue_PV<0, DCH>(dV0, tmem, idO, s, stV, n > 0);
                     if (!mbar_wait(smem_u32(&p_ready[2 * s + 1]), n & 1, p.timeout_ns, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    issue_PV(s, stV, true, 4);
+                    issue_PV<4, DCH>(dV0, tmem, idO, s, stV, true);
                     if (n == slot[s].n_kv - 1) mma_commit(smem_u32(&o_done[s]));
                     if (n + 1 < slot[s].n_kv) {
-                        issue_S(s, stK);
+                        issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
                         mma_commit(smem_u32(&s_full[s]));
                     }
                 }
