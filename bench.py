@@ -52,6 +52,9 @@ WORKLOADS = {
                             S=8192, d=128),
     "mqa_chunked_prefill_f16": dict(kind="cached", dtype="f16", B=32, H=8, Hkv=1, Tnew=512,
                                     start=3584, S=4096, d=128),
+    # the GQA decode over a paged cache: 64-token pages in a seeded physical order
+    "gqa_decode_paged_bf16": dict(kind="paged", dtype="bf16", B=64, H=32, Hkv=8, Tnew=1,
+                                  start=8191, S=8192, d=128, page=64),
     # the step before attention: the GQA prefill's 4096 new keys (RoPE) and values
     # written into an empty cache
     "kv_append_rope_gqa16x8_bf16": dict(kind="append", dtype="bf16", B=8, H=16, Hkv=8,
@@ -60,8 +63,10 @@ WORKLOADS = {
 DEFAULT_WORKLOAD = "bitnet3b_mha_prefill_bf16"
 DECODE_WORKLOAD = "gqa_decode_bf16"
 APPEND_WORKLOAD = "kv_append_rope_gqa16x8_bf16"
+PAGED_WORKLOAD = "gqa_decode_paged_bf16"
 TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
 KERNEL_SOURCES = {"tcgen05": "prefill_tcgen05.cuh", "splitkv": "decode_splitkv.cuh",
+                  "paged": "decode_splitkv.cuh",
                   "simt": "simt_attn.cuh", "append": "kv_append.cuh"}
 
 
@@ -107,7 +112,7 @@ def algorithmic_bytes(w):
 
 
 def bound(w):
-    if w["kind"] == "append":
+    if w["kind"] in ("append", "paged"):
         return "hbm"
     return "hbm" if w["kind"] == "cached" and q_len(w) * w["H"] // w["Hkv"] <= 16 else "tensor"
 
@@ -117,6 +122,9 @@ def config_of(name, w, world):
            "dtype": w["dtype"], "causal": True, "scale": f"1/sqrt({w['d']})"}
     if w["kind"] == "prefill":
         cfg["T"] = w["T"]
+    elif w["kind"] == "paged":
+        cfg.update(Tnew=w["Tnew"], kv_len=w["S"], page_size=w["page"],
+                   pages="seeded random physical order")
     elif w["kind"] == "append":
         cfg = {"workload": name, "B": w["B"], "Hkv": w["Hkv"], "d": w["d"], "dtype": w["dtype"],
                "Tnew": w["Tnew"], "start_pos": w["start"], "S_cap": w["S"],
@@ -262,6 +270,18 @@ class Case:
             self.kernel, self.launches, self.device = "append", 1, device
             return
         q, k, v = inputs.qkv(w["B"], w["H"], w["Hkv"], Tq, S, w["d"], dt, seed=seed)
+        if w["kind"] == "paged":
+            # pages [B * S / P, Hkv, P, d] in a seeded physical order, and the table
+            P, n = w["page"], S // w["page"]
+            perm = torch.randperm(w["B"] * n, generator=torch.Generator().manual_seed(seed))
+            def to_pages(t):
+                blocks = t.reshape(w["B"], w["Hkv"], n, P, w["d"]).permute(0, 2, 1, 3, 4)
+                pages = torch.empty((w["B"] * n, w["Hkv"], P, w["d"]), dtype=dt)
+                pages[perm] = blocks.reshape(w["B"] * n, w["Hkv"], P, w["d"])
+                return pages
+            k, v = to_pages(k), to_pages(v)
+            self.table = perm.reshape(w["B"], n).to(torch.int32).to(device)
+            self.lens = torch.full((w["B"],), S, dtype=torch.int32, device=device)
         self.host = [t.pin_memory() for t in (q, k, v)]
         self.q, self.k, self.v = (t.to(device, non_blocking=True) for t in self.host)
         self.out = torch.empty_like(self.q)
@@ -272,6 +292,10 @@ class Case:
         if w["kind"] == "prefill":
             self.kernel = attn.prefill_plan(dt, w["B"], w["H"], w["Hkv"], Tq, w["d"])
             self.ws = None
+        elif w["kind"] == "paged":
+            self.kernel = "splitkv"
+            need = attn.cached_paged_workspace_size(dt, w["B"], w["H"], w["Hkv"], Tq, w["d"], S)
+            self.ws = torch.empty(need, dtype=torch.uint8, device=device) if need else None
         else:
             self.kernel = attn.cached_plan(dt, w["B"], w["H"], w["Hkv"], Tq, S, S, w["d"],
                                            w["start"])
@@ -290,6 +314,9 @@ class Case:
                                      rope_base=w["base"])
         elif w["kind"] == "prefill":
             self.attn.prefill(self.q, self.k, self.v, scale=self.scale, causal=True, out=self.out)
+        elif w["kind"] == "paged":
+            self.attn.cached_paged(self.q, self.k, self.v, self.table, self.lens, max_kv_len=w["S"],
+                                   scale=self.scale, out=self.out, workspace=self.ws)
         else:
             self.attn.cached(self.q, self.k, self.v, start_pos=w["start"], scale=self.scale,
                              out=self.out, workspace=self.ws)
@@ -422,6 +449,11 @@ class OracleSample:
             self.v_new = inputs.normal(shape, seed, 2, dt)
             self.total = w["B"] * w["Tnew"]
             self.what = "(batch, token) rows of"
+        elif w["kind"] == "paged":
+            self.q, self.k, self.v = inputs.qkv(w["B"], w["H"], w["Hkv"], q_len(w), kv_len(w),
+                                                w["d"], dt, seed=seed)
+            self.total = w["B"]
+            self.what = "sequences (paged, all heads) of"
         else:
             self.q, self.k, self.v = inputs.qkv(w["B"], w["H"], w["Hkv"], q_len(w), kv_len(w),
                                                 w["d"], dt, seed=seed)
@@ -452,6 +484,24 @@ class OracleSample:
             for kn, vn, pos in jobs:
                 rope_append(kn, vn, start_pos=pos, base=w["base"])
             return time.perf_counter() - t0, n * self.per_unit, n
+        if w["kind"] == "paged":
+            from oracle import paged_attention
+
+            P, S = w["page"], kv_len(w)
+            secs = 0.0
+            for b in rng.choice(self.total, size=n, replace=False):
+                perm = torch.as_tensor(rng.permutation(S // P))
+                def pages(t):
+                    blocks = t[b].reshape(w["Hkv"], S // P, P, w["d"]).permute(1, 0, 2, 3)
+                    out = torch.empty_like(blocks)
+                    out[perm] = blocks
+                    return out
+                kp, vp = pages(self.k), pages(self.v)
+                t0 = time.perf_counter()
+                paged_attention(self.q[b:b + 1], kp, vp, perm.reshape(1, -1), [S],
+                                scale=1 / math.sqrt(w["d"]))
+                secs += time.perf_counter() - t0
+            return secs, n * self.per_unit, n
         rows = np.sort(rng.choice(self.total, size=n, replace=False))
         t0 = time.perf_counter()
         oracle_attention(self.q, self.k, self.v, scale=1 / math.sqrt(w["d"]), causal=True,
@@ -550,7 +600,8 @@ def run_ours(args, dist_ctx):
         "clocks": clocks,
         "device_status": status,
     }
-    legs = [] if args.no_decode else [("decode", DECODE_WORKLOAD), ("append", APPEND_WORKLOAD)]
+    legs = [] if args.no_decode else [("decode", DECODE_WORKLOAD), ("paged", PAGED_WORKLOAD),
+                                      ("append", APPEND_WORKLOAD)]
     del case
     for key, leg in legs:
         if leg == name:

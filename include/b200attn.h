@@ -44,7 +44,11 @@
  *   ATTN_ERR_WORKSPACE    workspace smaller than attn_cached_workspace_size();
  *   ATTN_ERR_CUDA         a CUDA runtime error while encoding or launching;
  *   ATTN_ERR_DEVICE_TIMEOUT reported by attn_device_status() when a kernel gave
- *                         up a bounded wait (it then exits cleanly).
+ *                         up a bounded wait (it then exits cleanly);
+ *   ATTN_ERR_DEVICE_INDEX reported by attn_device_status() when a paged call met
+ *                         a page table or length entry out of range (it clamps
+ *                         it and never reads outside the pools; that output is
+ *                         then meaningless).
  * A problem with B * H * Tq = 0 returns ATTN_OK and launches nothing.
  */
 #ifndef B200ATTN_H
@@ -69,7 +73,8 @@ typedef enum {
     ATTN_ERR_UNSUPPORTED = 2,
     ATTN_ERR_WORKSPACE = 3,
     ATTN_ERR_CUDA = 4,
-    ATTN_ERR_DEVICE_TIMEOUT = 5
+    ATTN_ERR_DEVICE_TIMEOUT = 5,
+    ATTN_ERR_DEVICE_INDEX = 6
 } attn_status_t;
 
 typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1, ATTN_F16 = 2 } attn_dtype_t;
@@ -160,6 +165,47 @@ ATTN_API attn_status_t attn_kv_append_rope(const void* k_new, const void* v_new,
                                            void* v_cache, attn_dtype_t dtype, int64_t B,
                                            int64_t Hkv, int64_t Tnew, int64_t S_cap, int64_t d,
                                            int64_t start_pos, float rope_base, void* stream);
+
+/*
+ * KV-cached attention over a paged cache: a logical-to-physical page table
+ * ("Causal Multi-Head Self-Attention", Algorithm and cache boundaries: paged
+ * decode reads a K/V page table; attention_cached.go, CausalAttentionPackedBlocks:
+ * head-major blocks [kv head][token within block][d]).  Same result as
+ * attn_cached on the gathered history, each sequence with its own length.
+ *   q [B,H,Tnew,d]; o [B,H,Tnew,d]; lse nullable [B,H,Tnew].  Always causal.
+ *   k_pages, v_pages [num_pages, Hkv, page_size, d]: page p holds, for every
+ *     K/V head, page_size consecutive tokens.
+ *   page_table (device, int32) [B, max_pages]: token j of sequence b lives in
+ *     physical page page_table[b][j / page_size], row j % page_size.
+ *   kv_lens (device, int32) [B]: L_b, the tokens of sequence b in the cache,
+ *     new ones included; its Tnew new tokens sit at positions L_b - Tnew ..
+ *     L_b - 1 and see keys 0 .. their own position.
+ *   max_kv_len (host): a bound on every L_b, used to plan the split; at most
+ *     max_pages * page_size.
+ *   page_size: a power of two, 8 .. 2^20.
+ *   workspace: at least attn_cached_paged_workspace_size() bytes, 16-byte
+ *     aligned; may be NULL when that size is 0.
+ * The device arrays are read, never written; entries out of range are
+ * reported through attn_device_status() as ATTN_ERR_DEVICE_INDEX.
+ * Supported: bf16 / fp16 with d in {64, 128} and H / Hkv * Tnew <= 16, or
+ * d = 256 and H / Hkv * Tnew <= 8 (the split-KV kernels); otherwise
+ * ATTN_ERR_UNSUPPORTED (float32 included).  ATTN_ERR_INVALID_ARG as for
+ * attn_cached, plus: page_size not a power of two in range, max_kv_len < Tnew
+ * or > max_pages * page_size, num_pages = 0, null or unaligned (4-byte) table
+ * or lengths.
+ */
+ATTN_API attn_status_t attn_cached_paged(const void* q, const void* k_pages, const void* v_pages,
+                                         void* o, float* lse, attn_dtype_t dtype, int64_t B,
+                                         int64_t H, int64_t Hkv, int64_t Tnew, int64_t d,
+                                         const int32_t* page_table, int64_t max_pages,
+                                         int64_t num_pages, int64_t page_size,
+                                         const int32_t* kv_lens, int64_t max_kv_len, float scale,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace attn_cached_paged needs (0 if none or unsupported). */
+ATTN_API size_t attn_cached_paged_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H,
+                                                 int64_t Hkv, int64_t Tnew, int64_t d,
+                                                 int64_t max_kv_len);
 
 /* Bytes of workspace attn_cached needs for this problem (0 if none).  Pure
  * host arithmetic; valid without a GPU.  Returns 0 for arguments that

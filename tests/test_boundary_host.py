@@ -56,7 +56,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings_and_version(lib):
     from transformer_attention_causal_b200 import _lib
 
-    for code in range(6):
+    for code in range(7):
         assert isinstance(_lib.status_string(code), str) and _lib.status_string(code)
     assert _lib.status_string(99) == "unknown status"
     assert lib.attn_version() >= 100
@@ -172,3 +172,36 @@ def test_append_limits_and_empty_calls(lib):
     # nothing to write: no launch, null pointers allowed
     assert append(lib, k=None, v=None, kc=None, vc=None, Tnew=0) == 0
     assert append(lib, k=None, v=None, kc=None, vc=None, B=0) == 0
+
+
+def paged(lib, q=FAKE, kp=FAKE, vp=FAKE, o=FAKE, dt=BF16, B=2, H=8, Hkv=2, Tnew=1, d=128,
+          table=ctypes.c_void_p(0x20000), max_pages=4, num_pages=8, page_size=16,
+          lens=ctypes.c_void_p(0x30000), max_kv_len=64, scale=0.1, ws=None, ws_bytes=0):
+    return lib.attn_cached_paged(q, kp, vp, o, None, dt, B, H, Hkv, Tnew, d, table, max_pages,
+                                 num_pages, page_size, lens, max_kv_len, scale, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kwargs", [
+    dict(table=None), dict(lens=None), dict(table=ctypes.c_void_p(0x20002)),
+    dict(page_size=12), dict(page_size=4), dict(page_size=0),
+    dict(max_kv_len=65),                 # > max_pages * page_size
+    dict(max_kv_len=0, Tnew=1),          # < Tnew
+    dict(num_pages=0), dict(q=None), dict(kp=MISALIGNED), dict(scale=float("nan")),
+    dict(H=6, Hkv=4), dict(dt=7),
+])
+def test_paged_rejects_invalid_arguments(lib, kwargs):
+    assert paged(lib, **kwargs) == INVALID
+
+
+def test_paged_limits(lib):
+    assert paged(lib, dt=F32) == UNSUPPORTED            # float32 has no split-KV kernel
+    assert paged(lib, H=32, Hkv=1, Tnew=1) == UNSUPPORTED   # 32 rows per K/V head
+    assert paged(lib, d=80) == UNSUPPORTED
+    # empty problems launch nothing
+    assert paged(lib, q=None, kp=None, vp=None, o=None, table=None, lens=None, B=0) == 0
+    # a split plan needs workspace
+    need = lib.attn_cached_paged_workspace_size(BF16, 64, 32, 8, 1, 128, 8192)
+    assert need > 0
+    assert paged(lib, B=64, H=32, Hkv=8, max_pages=128, num_pages=8192, page_size=64,
+                 max_kv_len=8192) == WORKSPACE
+    assert lib.attn_cached_paged_workspace_size(F32, 64, 32, 8, 1, 128, 8192) == 0

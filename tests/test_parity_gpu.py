@@ -148,6 +148,7 @@ CACHED_CASES = [
     (BF16, 2, 4, 4, 3, 497, 500, 500, 64, "splitkv"),       # MHA, 3 new tokens
     (BF16, 1, 4, 1, 4, 2900, 3000, 3100, 128, "splitkv"),   # history past the last query
     (F16, 2, 16, 2, 1, 4099, 4100, 4100, 256, "splitkv"),   # head size 256
+    (BF16, 2, 4, 4, 2, 1500, 1502, 1600, 256, "splitkv"),   # head size 256, two rows per K/V head
     (BF16, 1, 4, 1, 1, 19999, 20000, 20000, 128, "splitkv"),  # one long sequence: many splits
     (BF16, 2, 4, 2, 1, 0, 1, 1, 128, "splitkv"),            # first token
     (F16, 2, 8, 1, 200, 300, 500, 520, 128, "tcgen05"),     # MQA chunked prefill

@@ -16,8 +16,9 @@ import ctypes
 from . import _lib
 from ._lib import AttnError
 
-__all__ = ["prefill", "cached", "kv_append_rope", "cached_workspace_size", "prefill_plan",
-           "cached_plan", "device_status", "set_wait_timeout_ns", "AttnError"]
+__all__ = ["prefill", "cached", "cached_paged", "kv_append_rope", "cached_workspace_size",
+           "cached_paged_workspace_size", "prefill_plan", "cached_plan", "device_status",
+           "set_wait_timeout_ns", "AttnError"]
 
 
 def _torch():
@@ -109,6 +110,43 @@ def cached(q, k_hist, v_hist, *, start_pos: int, scale: float, S: int | None = N
                                  _stream_handle(stream, q.device))
     if st != _lib.OK:
         raise AttnError(st, "attn_cached")
+    return out
+
+
+def cached_paged_workspace_size(dtype, B, H, Hkv, Tnew, d, max_kv_len) -> int:
+    return int(_lib.load().attn_cached_paged_workspace_size(_code_of(dtype), B, H, Hkv, Tnew, d,
+                                                             max_kv_len))
+
+
+def cached_paged(q, k_pages, v_pages, page_table, kv_lens, *, max_kv_len: int, scale: float,
+                 out=None, lse=None, workspace=None, stream=None):
+    """New tokens of each sequence against its paged K/V history.
+    q [B,H,Tnew,d]; k_pages, v_pages [num_pages, Hkv, page_size, d];
+    page_table int32 [B, max_pages]; kv_lens int32 [B] (each sequence's length,
+    new tokens included; all <= max_kv_len)."""
+    torch = _torch()
+    _check(q, k_pages, v_pages, page_table, kv_lens, out, lse, workspace)
+    B, H, Tnew, d = q.shape
+    num_pages, Hkv, page_size = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    if tuple(v_pages.shape) != tuple(k_pages.shape) or k_pages.shape[3] != d:
+        raise ValueError("k_pages and v_pages must be [num_pages, Hkv, page_size, d] matching q")
+    if page_table.dtype != torch.int32 or kv_lens.dtype != torch.int32:
+        raise TypeError("page_table and kv_lens must be int32")
+    if page_table.dim() != 2 or page_table.shape[0] != B or tuple(kv_lens.shape) != (B,):
+        raise ValueError("page_table must be [B, max_pages] and kv_lens [B]")
+    if out is None:
+        out = q.new_empty(q.shape)
+    need = cached_paged_workspace_size(q.dtype, B, H, Hkv, Tnew, d, max_kv_len)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.load().attn_cached_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(out), _ptr(lse),
+                                       _dtype_code(q), B, H, Hkv, Tnew, d, _ptr(page_table),
+                                       page_table.shape[1], num_pages, page_size, _ptr(kv_lens),
+                                       int(max_kv_len), float(scale), _ptr(workspace), ws_bytes,
+                                       _stream_handle(stream, q.device))
+    if st != _lib.OK:
+        raise AttnError(st, "attn_cached_paged")
     return out
 
 

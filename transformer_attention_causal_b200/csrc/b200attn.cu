@@ -87,7 +87,8 @@ void plan_decode(const Problem& pb, Plan& pl) {
     const int64_t G = pb.H / pb.Hkv;
     pl.Rv = int(G * pb.Tq);
     pl.R = next_pow2_at_least4(pl.Rv);
-    pl.wide = (pl.R <= 8 && (pb.d == 64 || pb.d == 128)) || (pl.R == 4 && pb.d == 256);
+    // the wide kernel's three 120-key stages of K and V fit shared memory up to d = 128
+    pl.wide = pl.R <= 8 && (pb.d == 64 || pb.d == 128);
     const int stage_keys = pl.wide ? 120 : 64;
     const int ctas_per_sm = pl.wide ? 1 : 2;
     pl.kv_end = std::min<int64_t>(pb.S, pb.start_pos + pb.Tq);
@@ -224,10 +225,10 @@ attn_status_t run_simt(const Problem& pb, const void* q, const void* k, const vo
     return launch_status();
 }
 
-template <typename T, int D, int R>
-attn_status_t launch_decode_R(const DecodeParams& dp, cudaStream_t stream) {
+template <typename T, int D, int R, bool PAGED>
+attn_status_t launch_decode_RP(const DecodeParams& dp, cudaStream_t stream) {
     constexpr size_t smem = DecodeShape<D, R>::smem_bytes(sizeof(T));
-    auto kern = decode_splitkv_kernel<T, D, R>;
+    auto kern = decode_splitkv_kernel<T, D, R, PAGED>;
     static std::once_flag once[8];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -245,10 +246,10 @@ attn_status_t launch_decode_R(const DecodeParams& dp, cudaStream_t stream) {
     return ATTN_OK;
 }
 
-template <typename T, int D, int R>
-attn_status_t launch_decode_wide_R(const DecodeParams& dp, cudaStream_t stream) {
+template <typename T, int D, int R, bool PAGED>
+attn_status_t launch_decode_wide_RP(const DecodeParams& dp, cudaStream_t stream) {
     constexpr size_t smem = WideShape<D, R>::smem_bytes(sizeof(T));
-    auto kern = decode_wide_kernel<T, D, R>;
+    auto kern = decode_wide_kernel<T, D, R, PAGED>;
     static std::once_flag once[8];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -266,13 +267,28 @@ attn_status_t launch_decode_wide_R(const DecodeParams& dp, cudaStream_t stream) 
     return ATTN_OK;
 }
 
+template <typename T, int D, int R>
+attn_status_t launch_decode_R(const DecodeParams& dp, cudaStream_t stream) {
+    return dp.paged ? launch_decode_RP<T, D, R, true>(dp, stream)
+                    : launch_decode_RP<T, D, R, false>(dp, stream);
+}
+
+template <typename T, int D, int R>
+attn_status_t launch_decode_wide_R(const DecodeParams& dp, cudaStream_t stream) {
+    return dp.paged ? launch_decode_wide_RP<T, D, R, true>(dp, stream)
+                    : launch_decode_wide_RP<T, D, R, false>(dp, stream);
+}
+
 template <typename T, int D>
 attn_status_t launch_decode_D(int R, bool wide, const DecodeParams& dp, cudaStream_t stream) {
-    if (wide) {
-        if (R == 4) return launch_decode_wide_R<T, D, 4>(dp, stream);
-        if constexpr (D <= 128)
+    if constexpr (D <= 128) {
+        if (wide) {
+            if (R == 4) return launch_decode_wide_R<T, D, 4>(dp, stream);
             if (R == 8) return launch_decode_wide_R<T, D, 8>(dp, stream);
-        return ATTN_ERR_UNSUPPORTED;
+            return ATTN_ERR_UNSUPPORTED;
+        }
+    } else {
+        if (wide) return ATTN_ERR_UNSUPPORTED;
     }
     switch (R) {
     case 4: return launch_decode_R<T, D, 4>(dp, stream);
@@ -284,11 +300,19 @@ attn_status_t launch_decode_D(int R, bool wide, const DecodeParams& dp, cudaStre
     }
 }
 
+// A paged K/V cache: page pools, the page table and the per-sequence lengths.
+struct PagedKV {
+    const int32_t* page_table = nullptr;
+    const int32_t* kv_lens = nullptr;
+    int64_t max_pages = 0, num_pages = 0;
+    int page_shift = 0;
+};
+
 template <typename T>
 attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const void* k,
                          const void* v, void* o, float* lse, float scale, void* ws,
-                         cudaStream_t stream) {
-    DecodeParams dp;
+                         cudaStream_t stream, const PagedKV* paged = nullptr) {
+    DecodeParams dp{};
     dp.q = q; dp.k = k; dp.v = v; dp.o = o; dp.lse = lse;
     const size_t rows = size_t(pb.B * pb.Hkv) * pl.nsplit * pl.Rv;
     float* wsf = static_cast<float*>(ws);
@@ -302,6 +326,14 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
     dp.scale_log2 = scale * 1.4426950408889634f;
     dp.timeout_ns = g_timeout_ns.load();
     dp.test_flags = g_test_flags.load();
+    if (paged) {
+        dp.paged = 1;
+        dp.page_shift = paged->page_shift;
+        dp.page_table = paged->page_table;
+        dp.kv_lens = paged->kv_lens;
+        dp.max_pages = paged->max_pages;
+        dp.num_pages = paged->num_pages;
+    }
     switch (pb.d) {
     case 64: return launch_decode_D<T, 64>(pl.R, pl.wide, dp, stream);
     case 128: return launch_decode_D<T, 128>(pl.R, pl.wide, dp, stream);
@@ -476,6 +508,69 @@ attn_status_t attn_cached(const void* q, const void* k_hist, const void* v_hist,
                     static_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+// The problem a paged call plans as: every sequence at the host's length bound.
+Problem paged_problem(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t Tnew,
+                      int64_t d, int64_t max_kv_len) {
+    return Problem{dtype, B, H, Hkv, Tnew, max_kv_len, max_kv_len, d,
+                   max_kv_len - Tnew, 1, true};
+}
+
+}  // namespace
+
+attn_status_t attn_cached_paged(const void* q, const void* k_pages, const void* v_pages, void* o,
+                                float* lse, attn_dtype_t dtype, int64_t B, int64_t H,
+                                int64_t Hkv, int64_t Tnew, int64_t d, const int32_t* page_table,
+                                int64_t max_pages, int64_t num_pages, int64_t page_size,
+                                const int32_t* kv_lens, int64_t max_kv_len, float scale,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    if (!std::isfinite(scale) || max_kv_len < 0 || max_pages < 0 || num_pages < 0 || page_size < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_F16) {
+        if (dtype == ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+        return ATTN_ERR_INVALID_ARG;
+    }
+    if (B < 0 || H < 0 || Hkv < 0 || Tnew < 0 || d < 0) return ATTN_ERR_INVALID_ARG;
+    if (B == 0 || H == 0 || Tnew == 0) return ATTN_OK;
+    if (page_size < 8 || page_size > (int64_t(1) << 20) || (page_size & (page_size - 1)) != 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (max_kv_len < Tnew || max_kv_len > max_pages * page_size || num_pages == 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (!page_table || !kv_lens || !aligned4(page_table) || !aligned4(kv_lens))
+        return ATTN_ERR_INVALID_ARG;
+    const Problem pb = paged_problem(dtype, B, H, Hkv, Tnew, d, max_kv_len);
+    Plan pl;
+    attn_status_t st = make_plan(pb, pl);
+    if (st != ATTN_OK) return st;
+    if (pl.kernel != ATTN_KERNEL_SPLITKV) return ATTN_ERR_UNSUPPORTED;
+    st = check_pointers(pb, q, k_pages, v_pages, o, lse);
+    if (st != ATTN_OK) return st;
+    if (num_pages * Hkv * page_size * d > (int64_t(1) << 46)) return ATTN_ERR_UNSUPPORTED;
+    if (pl.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < pl.ws_bytes) return ATTN_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+    }
+    PagedKV pk;
+    pk.page_table = page_table;
+    pk.kv_lens = kv_lens;
+    pk.max_pages = max_pages;
+    pk.num_pages = num_pages;
+    while ((int64_t(1) << pk.page_shift) < page_size) ++pk.page_shift;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == ATTN_BF16)
+        return run_decode<__nv_bfloat16>(pb, pl, q, k_pages, v_pages, o, lse, scale, workspace, s, &pk);
+    return run_decode<__half>(pb, pl, q, k_pages, v_pages, o, lse, scale, workspace, s, &pk);
+}
+
+size_t attn_cached_paged_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                                        int64_t Tnew, int64_t d, int64_t max_kv_len) {
+    if (Tnew < 0 || max_kv_len < Tnew) return 0;
+    Plan pl;
+    if (make_plan(paged_problem(dtype, B, H, Hkv, Tnew, d, max_kv_len), pl) != ATTN_OK) return 0;
+    return pl.kernel == ATTN_KERNEL_SPLITKV ? pl.ws_bytes : 0;
+}
+
 size_t attn_cached_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
                                   int64_t Tnew, int64_t S, int64_t d, int64_t start_pos) {
     Problem pb{dtype, B, H, Hkv, Tnew, S, S, d, start_pos, 1, true};
@@ -509,6 +604,7 @@ const char* attn_status_string(attn_status_t status) {
     case ATTN_ERR_WORKSPACE: return "workspace too small";
     case ATTN_ERR_CUDA: return "CUDA runtime error";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a device-side wait timed out";
+    case ATTN_ERR_DEVICE_INDEX: return "a page table or length entry was out of range";
     }
     return "unknown status";
 }

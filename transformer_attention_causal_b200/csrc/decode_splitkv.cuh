@@ -47,7 +47,114 @@ struct DecodeParams {
     float scale_log2;    // scale * log2(e)
     uint64_t timeout_ns;
     uint32_t test_flags;  // kTestSkipLoads: issue no K/V copies (timeout-path tests)
+    // paged cache (paged != 0): k, v are page pools [num_pages, Hkv, 2^page_shift, D];
+    // page_table [B, max_pages] maps a sequence's logical page to a physical one;
+    // kv_lens [B] holds each sequence's length L_b (its new tokens at L_b - Tnew ..);
+    // S is then the host's bound on every L_b
+    int paged;
+    int page_shift;
+    const int32_t* page_table;
+    const int32_t* kv_lens;
+    int64_t max_pages, num_pages;
 };
+
+constexpr unsigned kStatusBadIndex = 6u;   // a page table or length entry out of range
+
+// Positions of a unit's rows: its new tokens start at `start_pos` and the
+// visible keys end at `kv_end`.  For a paged cache both come from the
+// sequence's own length; a length outside [Tnew, S] is recorded in the device
+// status word and clamped, so no load leaves the pool.
+__device__ __forceinline__ void decode_span(const DecodeParams& p, int b, int64_t& start_pos,
+                                            int64_t& kv_end) {
+    if (!p.paged) {
+        start_pos = p.start_pos;
+        kv_end = p.kv_end;
+        return;
+    }
+    int64_t L = p.kv_lens[b];
+    if (L < p.Tnew || L > p.S) {
+        atomicCAS(&g_device_status, 0u, kStatusBadIndex);
+        L = max64(p.Tnew, min64(L, p.S));
+    }
+    start_pos = L - p.Tnew;
+    kv_end = L;
+}
+
+// Issues the bulk copies of keys [k0, k0 + n) of (b, kv head) into kdst and
+// vdst, completing on `bar` (which expects 2 * n * D * sizeof(T) bytes).
+// Contiguous cache: one copy each, by lane 0.  Paged cache: the warp's lanes
+// read the page table entries the keys span (one each, so n must span at most
+// 32 pages) and lane 0 copies each page's run of rows; an entry outside the
+// pool is recorded and replaced by page 0, so no load leaves the pool.
+template <typename T, int D>
+__device__ __forceinline__ void load_kv_rows(const DecodeParams& p, int lane, int b, int kvh,
+                                             const T* kg, const T* vg, int64_t k0, int n,
+                                             T* kdst, T* vdst, uint32_t bar) {
+    if (!p.paged) {
+        if (lane == 0) {
+            const uint32_t bytes = uint32_t(n) * D * sizeof(T);
+            bulk_load(smem_u32(kdst), kg + k0 * D, bytes, bar);
+            bulk_load(smem_u32(vdst), vg + k0 * D, bytes, bar);
+        }
+        return;
+    }
+    const int64_t P = int64_t(1) << p.page_shift;
+    const int64_t first = k0 >> p.page_shift;
+    const int npg = int(((k0 + n - 1) >> p.page_shift) - first + 1);
+    int64_t phys = 0;
+    if (lane < npg) {
+        const int64_t lp = first + lane;
+        phys = lp < p.max_pages ? p.page_table[size_t(b) * p.max_pages + lp] : -1;
+        if (phys < 0 || phys >= p.num_pages) {
+            atomicCAS(&g_device_status, 0u, kStatusBadIndex);
+            phys = 0;
+        }
+    }
+    const T* kpool = static_cast<const T*>(p.k);
+    const T* vpool = static_cast<const T*>(p.v);
+    int off = 0;
+    for (int pg = 0; pg < npg; ++pg) {
+        const int64_t ph = __shfl_sync(0xffffffffu, phys, pg);
+        const int64_t j = k0 + off;
+        const int o = int(j & (P - 1));
+        const int seg = int(min64(P - o, int64_t(n - off)));
+        if (lane == 0) {
+            const size_t row = ((size_t(ph) * p.Hkv + kvh) * size_t(P) + o) * D;
+            const uint32_t bytes = uint32_t(seg) * D * sizeof(T);
+            bulk_load(smem_u32(kdst + size_t(off) * D), kpool + row, bytes, bar);
+            bulk_load(smem_u32(vdst + size_t(off) * D), vpool + row, bytes, bar);
+        }
+        off += seg;
+    }
+}
+
+// Producer for a contiguous cache (lane 0 alone): stage `it` holds keys
+// k_begin + it * TK .., K and V rows copied with one bulk copy each; full
+// barriers bars[0..NST), empty barriers bars[NST..2 NST).
+template <typename T, int D, int TK, int NST>
+__device__ __forceinline__ void producer_contiguous(const DecodeParams& p, int nstages,
+                                                    int64_t k_begin, int64_t k_end, const T* kg,
+                                                    const T* vg, T* ks, T* vs, uint64_t* bars,
+                                                    volatile int* abort_flag) {
+    int issued = 0;
+    const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : nstages;
+    for (int it = 0; it < n_loads; ++it) {
+        const int st = it % NST;
+        if (!mbar_wait(smem_u32(&bars[NST + st]), ((it / NST) & 1) ^ 1, p.timeout_ns, abort_flag))
+            break;
+        issued = it + 1;
+        const int64_t k0 = k_begin + int64_t(it) * TK;
+        const int n = int(min64(TK, k_end - k0));
+        const uint32_t bytes = uint32_t(n) * D * sizeof(T);
+        const uint32_t full = smem_u32(&bars[st]);
+        mbar_expect_tx(full, 2 * bytes);
+        bulk_load(smem_u32(ks + size_t(st) * TK * D), kg + k0 * D, bytes, full);
+        bulk_load(smem_u32(vs + size_t(st) * TK * D), vg + k0 * D, bytes, full);
+    }
+    // never leave while a copy into this CTA's shared memory is in flight
+    for (int it = issued - 1; it >= 0 && it >= issued - NST; --it)
+        mbar_wait(smem_u32(&bars[it % NST]), (it / NST) & 1, p.timeout_ns, nullptr);
+}
 
 template <int D, int R>
 struct DecodeShape {
@@ -75,7 +182,7 @@ struct DecodeShape {
     }
 };
 
-template <typename T, int D, int R>
+template <typename T, int D, int R, bool PAGED>
 __global__ void __launch_bounds__(160, 2)
 decode_splitkv_kernel(const DecodeParams p) {
     using Sh = DecodeShape<D, R>;
@@ -96,8 +203,10 @@ decode_splitkv_kernel(const DecodeParams p) {
     const int split = blockIdx.x;
     const int b = unit / p.Hkv;
     const int kvh = unit % p.Hkv;
+    int64_t start_pos = p.start_pos, kv_end = p.kv_end;
+    if constexpr (PAGED) decode_span(p, b, start_pos, kv_end);
     const int64_t k_begin = int64_t(split) * p.chunk;
-    const int64_t k_end = min(p.kv_end, k_begin + p.chunk);
+    const int64_t k_end = min64(kv_end, k_begin + p.chunk);
     const int nstages = k_end > k_begin ? int((k_end - k_begin + TK - 1) / TK) : 0;
 
     if (threadIdx.x == 0) {
@@ -114,28 +223,34 @@ decode_splitkv_kernel(const DecodeParams p) {
     const T* vg = static_cast<const T*>(p.v) + (size_t(unit) * p.S_cap) * D;
 
     if (warp == NW) {
-        // ------------------------------------------------ producer
-        if (lane == 0) {
-            int issued = 0;
-            const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : nstages;
-            for (int it = 0; it < n_loads; ++it) {
-                const int st = it % NST;
-                const uint32_t ph = (it / NST) & 1;
-                if (!mbar_wait(smem_u32(&bars[NST + st]), ph ^ 1, p.timeout_ns, abort_flag)) break;
-                issued = it + 1;
-                const int64_t k0 = k_begin + int64_t(it) * TK;
-                const int n = int(min64(TK, k_end - k0));
-                const uint32_t bytes = uint32_t(n) * D * sizeof(T);
-                const uint32_t full = smem_u32(&bars[st]);
-                mbar_expect_tx(full, 2 * bytes);
-                bulk_load(smem_u32(ks + size_t(st) * TK * D), kg + k0 * D, bytes, full);
-                bulk_load(smem_u32(vs + size_t(st) * TK * D), vg + k0 * D, bytes, full);
-            }
-            // Never leave while a copy into this CTA's shared memory is in
-            // flight: wait (bounded) for the last phase issued on each stage.
+        // ------------------------------------------------ producer (lane 0 waits
+        // and copies; for a paged cache the whole warp reads page table entries)
+        if constexpr (!PAGED) {
+            if (lane == 0) producer_contiguous<T, D, TK, NST>(p, nstages, k_begin, k_end, kg, vg, ks, vs,
+                                                              bars, abort_flag);
+            return;
+        }
+        int issued = 0;
+        const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : nstages;
+        for (int it = 0; it < n_loads; ++it) {
+            const int st = it % NST;
+            const uint32_t ph = (it / NST) & 1;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(smem_u32(&bars[NST + st]), ph ^ 1, p.timeout_ns, abort_flag);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            issued = it + 1;
+            const int64_t k0 = k_begin + int64_t(it) * TK;
+            const int n = int(min64(TK, k_end - k0));
+            const uint32_t full = smem_u32(&bars[st]);
+            if (lane == 0) mbar_expect_tx(full, 2 * uint32_t(n) * D * sizeof(T));
+            load_kv_rows<T, D>(p, lane, b, kvh, kg, vg, k0, n, ks + size_t(st) * TK * D,
+                               vs + size_t(st) * TK * D, full);
+        }
+        // Never leave while a copy into this CTA's shared memory is in
+        // flight: wait (bounded) for the last phase issued on each stage.
+        if (lane == 0)
             for (int it = issued - 1; it >= 0 && it >= issued - NST; --it)
                 mbar_wait(smem_u32(&bars[it % NST]), (it / NST) & 1, p.timeout_ns, nullptr);
-        }
         return;
     }
 
@@ -165,7 +280,7 @@ decode_splitkv_kernel(const DecodeParams p) {
     int64_t row_lim[R];
 #pragma unroll
     for (int r = 0; r < R; ++r)
-        row_lim[r] = (r < p.Rv) ? p.start_pos + (r % p.Tnew) : -1;
+        row_lim[r] = (r < p.Rv) ? start_pos + (r % p.Tnew) : -1;
 
     float oacc[R][NCH][CE];
 #pragma unroll
@@ -512,7 +627,7 @@ __device__ __forceinline__ void load_elems(const T* src, float (&f)[N]) {
     }
 }
 
-template <typename T, int D, int R>
+template <typename T, int D, int R, bool PAGED>
 __global__ void __launch_bounds__(512, 1)
 decode_wide_kernel(const DecodeParams p) {
     using Sh = WideShape<D, R>;
@@ -532,8 +647,10 @@ decode_wide_kernel(const DecodeParams p) {
     const int split = blockIdx.x;
     const int b = unit / p.Hkv;
     const int kvh = unit % p.Hkv;
+    int64_t start_pos = p.start_pos, kv_end = p.kv_end;
+    if constexpr (PAGED) decode_span(p, b, start_pos, kv_end);
     const int64_t k_begin = int64_t(split) * p.chunk;
-    const int64_t k_end = min64(p.kv_end, k_begin + p.chunk);
+    const int64_t k_end = min64(kv_end, k_begin + p.chunk);
     const int nstages = k_end > k_begin ? int((k_end - k_begin + TK - 1) / TK) : 0;
 
     if (threadIdx.x == 0) {
@@ -550,25 +667,30 @@ decode_wide_kernel(const DecodeParams p) {
     const T* vg = static_cast<const T*>(p.v) + (size_t(unit) * p.S_cap) * D;
 
     if (warp == NW) {
-        if (lane == 0) {
-            int issued = 0;
-            const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : nstages;
-            for (int it = 0; it < n_loads; ++it) {
-                const int st = it % NST;
-                if (!mbar_wait(smem_u32(&bars[NST + st]), ((it / NST) & 1) ^ 1, p.timeout_ns, abort_flag))
-                    break;
-                issued = it + 1;
-                const int64_t k0 = k_begin + int64_t(it) * TK;
-                const int n = int(min64(TK, k_end - k0));
-                const uint32_t bytes = uint32_t(n) * D * sizeof(T);
-                const uint32_t full = smem_u32(&bars[st]);
-                mbar_expect_tx(full, 2 * bytes);
-                bulk_load(smem_u32(ks + size_t(st) * TK * D), kg + k0 * D, bytes, full);
-                bulk_load(smem_u32(vs + size_t(st) * TK * D), vg + k0 * D, bytes, full);
-            }
+        if constexpr (!PAGED) {
+            if (lane == 0) producer_contiguous<T, D, TK, NST>(p, nstages, k_begin, k_end, kg, vg, ks, vs,
+                                                              bars, abort_flag);
+            return;
+        }
+        int issued = 0;
+        const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : nstages;
+        for (int it = 0; it < n_loads; ++it) {
+            const int st = it % NST;
+            bool ok = true;
+            if (lane == 0)
+                ok = mbar_wait(smem_u32(&bars[NST + st]), ((it / NST) & 1) ^ 1, p.timeout_ns, abort_flag);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            issued = it + 1;
+            const int64_t k0 = k_begin + int64_t(it) * TK;
+            const int n = int(min64(TK, k_end - k0));
+            const uint32_t full = smem_u32(&bars[st]);
+            if (lane == 0) mbar_expect_tx(full, 2 * uint32_t(n) * D * sizeof(T));
+            load_kv_rows<T, D>(p, lane, b, kvh, kg, vg, k0, n, ks + size_t(st) * TK * D,
+                               vs + size_t(st) * TK * D, full);
+        }
+        if (lane == 0)
             for (int it = issued - 1; it >= 0 && it >= issued - NST; --it)
                 mbar_wait(smem_u32(&bars[it % NST]), (it / NST) & 1, p.timeout_ns, nullptr);
-        }
         return;
     }
 
@@ -602,7 +724,7 @@ decode_wide_kernel(const DecodeParams p) {
     const bool single = p.Tnew == 1;  // every key below kv_end is visible
     int64_t row_lim[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) row_lim[r] = (r < p.Rv) ? p.start_pos + (r % p.Tnew) : -1;
+    for (int r = 0; r < R; ++r) row_lim[r] = (r < p.Rv) ? start_pos + (r % p.Tnew) : -1;
 
     float2 o2[R][EC / 2];
 #pragma unroll
