@@ -51,6 +51,10 @@ def _bind(path: str):
     lib.oracle_attention.argtypes = [vp, vp, vp, ctypes.c_int, i64, i64, i64, i64, i64,
                                      i64, i64, i64, dbl, ctypes.c_int, vp, i64, vp, vp,
                                      vp, ctypes.c_int]
+    lib.oracle_attention_window.restype = ctypes.c_int
+    lib.oracle_attention_window.argtypes = [vp, vp, vp, ctypes.c_int, i64, i64, i64, i64, i64,
+                                            i64, i64, i64, dbl, ctypes.c_int, i64, vp, i64, vp,
+                                            vp, vp, ctypes.c_int]
     lib.oracle_widen_bf16.restype = dbl
     lib.oracle_widen_bf16.argtypes = [ctypes.c_uint16]
     lib.oracle_widen_f16.restype = dbl
@@ -106,11 +110,12 @@ def _as_raw(x):
 
 def attention(q, k, v, *, scale: float, causal: bool = True, start_pos: int = 0,
               S: int | None = None, rows=None, want_lse: bool = False,
-              want_probs: bool = False, nthreads: int = 0, _lib_handle=None):
+              want_probs: bool = False, nthreads: int = 0, window: int = 0, _lib_handle=None):
     """fp64 attention rows.
 
     q: [B, H, Tq, d]; k, v: [B, Hkv, S_cap, d] (first ``S`` rows valid; default
     S = S_cap).  Query row i sits at absolute position ``start_pos + i``.
+    ``window`` w > 0 keeps only keys p - w < j <= p (a local window).
     ``rows``: optional iterable of flat row ids ``(b*H + h)*Tq + i``; the
     result then has one row per id, in that order.
 
@@ -143,10 +148,10 @@ def attention(q, k, v, *, scale: float, causal: bool = True, start_pos: int = 0,
     probs = np.zeros((nrows, S), dtype=np.float64) if want_probs else None
     ptr = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
     lib = _lib() if _lib_handle is None else _lib_handle
-    rc = lib.oracle_attention(
+    rc = lib.oracle_attention_window(
         ptr(qa), ptr(ka), ptr(va), code, B, H, Hkv, Tq, S, S_cap, d, int(start_pos),
-        float(scale), int(bool(causal)), ptr(rows_arr), nrows, ptr(out), ptr(lse), ptr(probs),
-        int(nthreads))
+        float(scale), int(bool(causal)), int(window), ptr(rows_arr), nrows, ptr(out), ptr(lse),
+        ptr(probs), int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_attention rejected its arguments (code {rc})")
     res = [out.reshape(out_shape)]

@@ -15,9 +15,12 @@
  *   p    = start_pos + i                          absolute position of query i
  *        ("makarna attention_cached.go" CausalAttentionCached: new tokens start
  *         at startPos, the history holds every earlier and current key)
- *   vis  = { j < S : !causal or j <= p }          causal mask: 0 on and below the
- *        diagonal, -inf above ("Hesper.Layers.Attention" Causal Masking;
- *        "Grouped-Query Attention" §5.2)
+ *   vis  = { j < S : (!causal or j <= p) and (window = 0 or j > p - window) }
+ *        causal mask: 0 on and below the diagonal, -inf above
+ *        ("Hesper.Layers.Attention" Causal Masking; "Grouped-Query Attention"
+ *        §5.2); a local window of w keys keeps only the current position and
+ *        the previous w - 1 ("Multi-query attention, annotated" §4.1: local
+ *        versions attend to the current position and the previous 31)
  *   s_j  = scale * sum_t Q[b,h,i,t] * K[b,kvh,j,t]   for j in vis
  *        (scores = Q K^T / sqrt(d_k): "Hesper.Layers.Attention" Mathematical
  *         Definition; the scale is an explicit argument because the worked
@@ -87,12 +90,20 @@ typedef struct {
     int64_t B, H, Hkv, Tq, S, S_cap, d, start_pos;
     double scale;
     int causal;
+    int64_t window; /* 0: no window */
     const int64_t* rows;
     int64_t nrows;
     double *out, *lse, *probs;
     int64_t first, last; /* half-open range of requested rows for one worker */
     int status;
 } job_t;
+
+/* Is key j visible to the query at absolute position p? */
+static int visible(const job_t* J, int64_t j, int64_t p) {
+    if (J->causal && j > p) return 0;
+    if (J->window > 0 && j <= p - J->window) return 0;
+    return 1;
+}
 
 /* One output row, straight from the definition in the file header. */
 static int one_row(const job_t* J, int64_t slot, double* s, double* w) {
@@ -111,8 +122,7 @@ static int one_row(const job_t* J, int64_t slot, double* s, double* w) {
     /* visible keys and their scores */
     int64_t nvis = 0;
     for (int64_t j = 0; j < J->S; ++j) {
-        int visible = !J->causal || j <= p;
-        if (!visible) continue;
+        if (!visible(J, j, p)) continue;
         double dot = 0.0;
         for (int64_t t = 0; t < d; ++t)
             dot += load_elem(J->q, J->dtype, q_off + t) *
@@ -134,19 +144,19 @@ static int one_row(const job_t* J, int64_t slot, double* s, double* w) {
     /* pass 1: maximum over the visible scores */
     double M = -INFINITY;
     for (int64_t j = 0; j < J->S; ++j) {
-        if (J->causal && j > p) continue;
+        if (!visible(J, j, p)) continue;
         if (s[j] > M) M = s[j];
     }
     /* pass 2: exponentials and their sum */
     double L = 0.0;
     for (int64_t j = 0; j < J->S; ++j) {
-        if (J->causal && j > p) { w[j] = 0.0; continue; }
+        if (!visible(J, j, p)) { w[j] = 0.0; continue; }
         w[j] = exp(s[j] - M);
         L += w[j];
     }
     /* weighted sum of the visible value rows */
     for (int64_t j = 0; j < J->S; ++j) {
-        if (J->causal && j > p) continue;
+        if (!visible(J, j, p)) continue;
         double pj = w[j] / L;
         if (J->probs) J->probs[slot * J->S + j] = pj;
         for (int64_t t = 0; t < d; ++t)
@@ -174,13 +184,13 @@ static void* worker(void* arg) {
  * nthreads <= 0 uses every online core.  Returns 0, or a negative code on a
  * malformed argument (checked here so the tests can rely on it).
  */
-int oracle_attention(const void* q, const void* k, const void* v, int dtype,
-                     int64_t B, int64_t H, int64_t Hkv, int64_t Tq, int64_t S,
-                     int64_t S_cap, int64_t d, int64_t start_pos, double scale,
-                     int causal, const int64_t* rows, int64_t nrows, double* out,
-                     double* lse, double* probs, int nthreads) {
+int oracle_attention_window(const void* q, const void* k, const void* v, int dtype,
+                            int64_t B, int64_t H, int64_t Hkv, int64_t Tq, int64_t S,
+                            int64_t S_cap, int64_t d, int64_t start_pos, double scale,
+                            int causal, int64_t window, const int64_t* rows, int64_t nrows,
+                            double* out, double* lse, double* probs, int nthreads) {
     if (B < 0 || H <= 0 || Hkv <= 0 || H % Hkv || Tq < 0 || S < 0 || S_cap < S ||
-        d <= 0 || start_pos < 0 || dtype < 0 || dtype > 3)
+        d <= 0 || start_pos < 0 || dtype < 0 || dtype > 3 || window < 0)
         return -1;
     int64_t total = B * H * Tq;
     if (!rows) nrows = total;
@@ -202,6 +212,7 @@ int oracle_attention(const void* q, const void* k, const void* v, int dtype,
         J->q = q; J->k = k; J->v = v; J->dtype = dtype;
         J->B = B; J->H = H; J->Hkv = Hkv; J->Tq = Tq; J->S = S; J->S_cap = S_cap;
         J->d = d; J->start_pos = start_pos; J->scale = scale; J->causal = causal;
+        J->window = window;
         J->rows = rows; J->nrows = nrows; J->out = out; J->lse = lse; J->probs = probs;
         J->first = nrows * t / nthreads;
         J->last = nrows * (t + 1) / nthreads;
@@ -271,4 +282,14 @@ int oracle_rope_append(const void* k_new, const void* v_new, int dtype, int64_t 
                 }
             }
     return 0;
+}
+
+/* The same without a local window. */
+int oracle_attention(const void* q, const void* k, const void* v, int dtype,
+                     int64_t B, int64_t H, int64_t Hkv, int64_t Tq, int64_t S,
+                     int64_t S_cap, int64_t d, int64_t start_pos, double scale,
+                     int causal, const int64_t* rows, int64_t nrows, double* out,
+                     double* lse, double* probs, int nthreads) {
+    return oracle_attention_window(q, k, v, dtype, B, H, Hkv, Tq, S, S_cap, d, start_pos, scale,
+                                   causal, 0, rows, nrows, out, lse, probs, nthreads);
 }

@@ -2,7 +2,8 @@
 
 Each case compiles a copy of ``oracle/attn_oracle.c`` with one deliberate
 mistake planted in it (on the CPU, into a temporary directory) and runs every
-pin of ``test_oracle_pins.py`` and ``test_oracle_rope_pins.py`` against that
+pin of ``test_oracle_pins.py``, ``test_oracle_rope_pins.py`` and
+``test_oracle_window_pins.py`` against that
 copy: at least one pin must fail.
 The unmodified oracle passes all of them (that file's own run).
 """
@@ -14,6 +15,7 @@ import pytest
 
 import test_oracle_pins as pins
 import test_oracle_rope_pins as rope_pins
+import test_oracle_window_pins as window_pins
 from oracle.attention import load_variant
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle",
@@ -22,10 +24,12 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), 
 # (name, [(exact text in attn_oracle.c, replacement), ...])
 MUTANTS = [
     ("scale dropped", [("s[j] = J->scale * dot;", "s[j] = dot;")]),
-    ("mask includes diagonal off by one", [("!J->causal || j <= p", "!J->causal || j < p"),
-                                          ("J->causal && j > p", "J->causal && j >= p")]),
-    ("mask one position too wide", [("!J->causal || j <= p", "!J->causal || j <= p + 1"),
-                                    ("J->causal && j > p", "J->causal && j > p + 1")]),
+    ("mask includes diagonal off by one", [("if (J->causal && j > p) return 0;",
+                                           "if (J->causal && j >= p) return 0;")]),
+    ("mask one position too wide", [("if (J->causal && j > p) return 0;",
+                                     "if (J->causal && j > p + 1) return 0;")]),
+    ("window one key too wide", [("j <= p - J->window) return 0;", "j < p - J->window) return 0;")]),
+    ("window ignored", [("if (J->window > 0 && j <= p - J->window) return 0;", "")]),
     ("GQA head taken modulo", [("int64_t kvh = h / g;", "int64_t kvh = h % J->Hkv;")]),
     ("start_pos ignored", [("int64_t p = J->start_pos + i;", "int64_t p = i;")]),
     ("exponent sign flipped", [("w[j] = exp(s[j] - M);", "w[j] = exp(M - s[j]);")]),
@@ -56,7 +60,8 @@ def _pin_calls(golden_dir):
     """Every test function of the pin modules, with its parameter sets."""
     calls = []
     members = inspect.getmembers(pins, inspect.isfunction) + \
-        inspect.getmembers(rope_pins, inspect.isfunction)
+        inspect.getmembers(rope_pins, inspect.isfunction) + \
+        inspect.getmembers(window_pins, inspect.isfunction)
     for name, fn in members:
         if not name.startswith("test_"):
             continue
@@ -91,6 +96,7 @@ def test_planted_mistake_fails_a_pin(name, edits, tmp_path, golden_dir, monkeypa
     monkeypatch.setattr(pins, "attention", variant.attention)
     monkeypatch.setattr(pins, "widen_bits", variant.widen_bits)
     monkeypatch.setattr(rope_pins, "rope_append", variant.rope_append)
+    monkeypatch.setattr(window_pins, "attention", variant.attention)
     failed = []
     for test_name, fn, kwargs in _pin_calls(golden_dir):
         try:
