@@ -6,9 +6,11 @@
 One step = one call of the library on one batch of the workload (default: the
 BitNet-3B-shaped causal MHA prefill, B=1, H=32, T=2048, d=80, bf16).  The
 line also carries the cached-decode half of the metric (GQA decode, B=64,
-H=32/8, S=8192, d=128, bf16) and the KV-cache append with RoPE on K of the
-GQA prefill's keys and values (B=8, Hkv=8, 4096 tokens, d=128, bf16), each
-measured the same way with its own roofline.
+H=32/8, S=8192, d=128, bf16), the same decode over a paged cache (64-token
+pages), the GQA prefill with a 2048-key local window (B=2, T=8192), and the
+KV-cache append with RoPE on K of the GQA prefill's keys and values (B=8,
+Hkv=8, 4096 tokens, d=128, bf16), each measured the same way with its own
+roofline.
 
 Timing: W untimed steps, then exactly K timed steps bracketed by a barrier and
 torch.cuda.synchronize() on both sides.  Before every timed call L2 is flushed
@@ -48,6 +50,9 @@ WORKLOADS = {
     "bitnet3b_mha_prefill_bf16": dict(kind="prefill", dtype="bf16", B=1, H=32, Hkv=32, T=2048,
                                       d=80),
     "gqa16x8_prefill_bf16": dict(kind="prefill", dtype="bf16", B=8, H=16, Hkv=8, T=4096, d=128),
+    # local attention: the GQA shape over 8192 tokens with a 2048-key window
+    "gqa_prefill_swa_bf16": dict(kind="prefill", dtype="bf16", B=2, H=32, Hkv=8, T=8192, d=128,
+                                 window=2048),
     "gqa_decode_bf16": dict(kind="cached", dtype="bf16", B=64, H=32, Hkv=8, Tnew=1, start=8191,
                             S=8192, d=128),
     "mqa_chunked_prefill_f16": dict(kind="cached", dtype="f16", B=32, H=8, Hkv=1, Tnew=512,
@@ -63,6 +68,7 @@ WORKLOADS = {
 DEFAULT_WORKLOAD = "bitnet3b_mha_prefill_bf16"
 DECODE_WORKLOAD = "gqa_decode_bf16"
 APPEND_WORKLOAD = "kv_append_rope_gqa16x8_bf16"
+WINDOW_WORKLOAD = "gqa_prefill_swa_bf16"
 PAGED_WORKLOAD = "gqa_decode_paged_bf16"
 TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
 KERNEL_SOURCES = {"tcgen05": "prefill_tcgen05.cuh", "splitkv": "decode_splitkv.cuh",
@@ -85,8 +91,12 @@ def start_pos(w):
 
 
 def visible_pairs(w):
-    """Visible (query, key) pairs per query head: sum over rows of (p_i + 1)."""
+    """Visible (query, key) pairs per query head: sum over rows of (p_i + 1),
+    or of min(p_i + 1, window) with a local window."""
     Tq, s0 = q_len(w), start_pos(w)
+    win = w.get("window", 0)
+    if win:
+        return sum(min(s0 + i + 1, win) for i in range(Tq))
     return Tq * s0 + Tq * (Tq + 1) // 2
 
 
@@ -122,6 +132,8 @@ def config_of(name, w, world):
            "dtype": w["dtype"], "causal": True, "scale": f"1/sqrt({w['d']})"}
     if w["kind"] == "prefill":
         cfg["T"] = w["T"]
+        if w.get("window"):
+            cfg["window"] = w["window"]
     elif w["kind"] == "paged":
         cfg.update(Tnew=w["Tnew"], kv_len=w["S"], page_size=w["page"],
                    pages="seeded random physical order")
@@ -313,7 +325,8 @@ class Case:
             self.attn.kv_append_rope(*self.dev_in, *self.dev_out, start_pos=w["start"],
                                      rope_base=w["base"])
         elif w["kind"] == "prefill":
-            self.attn.prefill(self.q, self.k, self.v, scale=self.scale, causal=True, out=self.out)
+            self.attn.prefill(self.q, self.k, self.v, scale=self.scale, causal=True, out=self.out,
+                              window=w.get("window", 0))
         elif w["kind"] == "paged":
             self.attn.cached_paged(self.q, self.k, self.v, self.table, self.lens, max_kv_len=w["S"],
                                    scale=self.scale, out=self.out, workspace=self.ws)
@@ -505,12 +518,14 @@ class OracleSample:
         rows = np.sort(rng.choice(self.total, size=n, replace=False))
         t0 = time.perf_counter()
         oracle_attention(self.q, self.k, self.v, scale=1 / math.sqrt(w["d"]), causal=True,
-                         start_pos=start_pos(w), rows=rows)
+                         start_pos=start_pos(w), rows=rows, window=w.get("window", 0))
         secs = time.perf_counter() - t0
         if self.unit == "GB/s":
             return secs, n * self.per_unit, n
-        i = rows % q_len(w)
-        return secs, float(np.sum(4 * w["d"] * (start_pos(w) + i + 1))) / 1e12, n
+        vis = start_pos(w) + rows % q_len(w) + 1
+        if w.get("window"):
+            vis = np.minimum(vis, w["window"])
+        return secs, float(np.sum(4 * w["d"] * vis)) / 1e12, n
 
     def sized(self, target_s, rng):
         """Rows that take the oracle about target_s seconds, from a pilot run."""
@@ -601,7 +616,7 @@ def run_ours(args, dist_ctx):
         "device_status": status,
     }
     legs = [] if args.no_decode else [("decode", DECODE_WORKLOAD), ("paged", PAGED_WORKLOAD),
-                                      ("append", APPEND_WORKLOAD)]
+                                      ("window", WINDOW_WORKLOAD), ("append", APPEND_WORKLOAD)]
     del case
     for key, leg in legs:
         if leg == name:
@@ -612,10 +627,12 @@ def run_ours(args, dist_ctx):
         lsteps = max(args.steps, 5)
         l_ms, _ = time_device(lcase, lsteps, max(args.warmup, 3), dist_ctx)
         l_ms = dist_ctx.max(l_ms)
+        hbm = bound(wl) == "hbm"
+        work = algorithmic_bytes(wl) / 1e9 if hbm else algorithmic_flops(wl) / 1e12
         line[key] = {
             "workload": leg,
-            "value": round(N * algorithmic_bytes(wl) / 1e9 / (l_ms * 1e-3), 2),
-            "unit": "GB/s", "ms_per_step": round(l_ms, 5), "steps": lsteps,
+            "value": round(N * work / (l_ms * 1e-3), 2),
+            "unit": "GB/s" if hbm else "TFLOP/s", "ms_per_step": round(l_ms, 5), "steps": lsteps,
             "gpu_launches": lsteps * lcase.launches,
             "roofline": roofline(wl, l_ms, lcase.kernel, leg, peaks, peak_src),
         }

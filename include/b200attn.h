@@ -167,6 +167,31 @@ ATTN_API attn_status_t attn_kv_append_rope(const void* k_new, const void* v_new,
                                            int64_t start_pos, float rope_base, void* stream);
 
 /*
+ * Local (sliding-window) attention: the query at absolute position p sees
+ * only keys p - window < j <= p, the current position and the previous
+ * window - 1 ("Multi-query attention, annotated" §4.1: local decoder
+ * self-attention over the current position and the previous 31).  Otherwise
+ * identical to attn_prefill (causal) and attn_cached; window = 0 is plain
+ * causal attention.  Key tiles wholly outside every row's window are never
+ * loaded.  Errors as for those calls, plus ATTN_ERR_INVALID_ARG for window < 0.
+ * attn_cached_local needs attn_cached_local_workspace_size() bytes of
+ * workspace (the split plan covers only the keys inside the window).
+ */
+ATTN_API attn_status_t attn_prefill_local(const void* q, const void* k, const void* v, void* o,
+                                          float* lse, attn_dtype_t dtype, int64_t B, int64_t H,
+                                          int64_t Hkv, int64_t T, int64_t d, float scale,
+                                          int64_t window, void* stream);
+ATTN_API attn_status_t attn_cached_local(const void* q, const void* k_hist, const void* v_hist,
+                                         void* o, float* lse, attn_dtype_t dtype, int64_t B,
+                                         int64_t H, int64_t Hkv, int64_t Tnew, int64_t S,
+                                         int64_t S_cap, int64_t d, int64_t start_pos, float scale,
+                                         int64_t window, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+ATTN_API size_t attn_cached_local_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H,
+                                                 int64_t Hkv, int64_t Tnew, int64_t S, int64_t d,
+                                                 int64_t start_pos, int64_t window);
+
+/*
  * KV-cached attention over a paged cache: a logical-to-physical page table
  * ("Causal Multi-Head Self-Attention", Algorithm and cache boundaries: paged
  * decode reads a K/V page table; attention_cached.go, CausalAttentionPackedBlocks:

@@ -24,6 +24,14 @@ def test_visible_pairs_match_a_mask_count(Tq, S, start):
     assert bench.visible_pairs(w) == brute_visible_pairs(Tq, S, start)
 
 
+@pytest.mark.parametrize("Tq,S,start,win", [(16, 16, 0, 4), (7, 30, 23, 10), (40, 40, 0, 64)])
+def test_windowed_visible_pairs_match_a_mask_count(Tq, S, start, win):
+    w = dict(kind="cached", Tnew=Tq, S=S, start=start, window=win)
+    i = np.arange(Tq)[:, None] + start
+    j = np.arange(S)[None, :]
+    assert bench.visible_pairs(w) == int(((j <= i) & (j > i - win)).sum())
+
+
 def test_workload_work_figures():
     W = bench.WORKLOADS
     # 4*d FLOPs per visible pair per query head

@@ -64,9 +64,11 @@ def _check(*tensors):
             raise ValueError("tensors must be contiguous")
 
 
-def prefill(q, k, v, *, scale: float, causal: bool = True, out=None, lse=None, stream=None):
+def prefill(q, k, v, *, scale: float, causal: bool = True, out=None, lse=None, stream=None,
+            window: int = 0):
     """Full-sequence attention.  q [B,H,T,d]; k, v [B,Hkv,T,d]; returns O [B,H,T,d].
-    ``lse`` (optional float32 [B,H,T]) receives the log-sum-exp of each row."""
+    ``lse`` (optional float32 [B,H,T]) receives the log-sum-exp of each row.
+    ``window`` w > 0: local attention, row p sees keys p - w < j <= p (causal)."""
     _check(q, k, v, out, lse)
     B, H, T, d = q.shape
     Hkv = k.shape[1]
@@ -74,6 +76,15 @@ def prefill(q, k, v, *, scale: float, causal: bool = True, out=None, lse=None, s
         raise ValueError("k and v must be [B, Hkv, T, d] matching q")
     if out is None:
         out = q.new_empty(q.shape)
+    if window:
+        if not causal:
+            raise ValueError("a local window is causal")
+        st = _lib.load().attn_prefill_local(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                            _dtype_code(q), B, H, Hkv, T, d, float(scale),
+                                            int(window), _stream_handle(stream, q.device))
+        if st != _lib.OK:
+            raise AttnError(st, "attn_prefill_local")
+        return out
     st = _lib.load().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _dtype_code(q),
                                   B, H, Hkv, T, d, float(scale), int(bool(causal)),
                                   _stream_handle(stream, q.device))
@@ -82,13 +93,16 @@ def prefill(q, k, v, *, scale: float, causal: bool = True, out=None, lse=None, s
     return out
 
 
-def cached_workspace_size(dtype, B, H, Hkv, Tnew, S, d, start_pos) -> int:
+def cached_workspace_size(dtype, B, H, Hkv, Tnew, S, d, start_pos, window: int = 0) -> int:
+    if window:
+        return int(_lib.load().attn_cached_local_workspace_size(_code_of(dtype), B, H, Hkv, Tnew,
+                                                                 S, d, start_pos, window))
     return int(_lib.load().attn_cached_workspace_size(_code_of(dtype), B, H, Hkv, Tnew, S, d,
                                                        start_pos))
 
 
 def cached(q, k_hist, v_hist, *, start_pos: int, scale: float, S: int | None = None, out=None,
-           lse=None, workspace=None, stream=None):
+           lse=None, workspace=None, stream=None, window: int = 0):
     """New tokens at ``start_pos`` against a K/V history that already holds them.
     q [B,H,Tnew,d]; k_hist, v_hist [B,Hkv,S_cap,d] (first S rows valid, default
     S = S_cap).  ``workspace`` (uint8 CUDA tensor) is allocated here when not given."""
@@ -100,10 +114,19 @@ def cached(q, k_hist, v_hist, *, start_pos: int, scale: float, S: int | None = N
     S = S_cap if S is None else int(S)
     if out is None:
         out = q.new_empty(q.shape)
-    need = cached_workspace_size(q.dtype, B, H, Hkv, Tnew, S, d, start_pos)
+    need = cached_workspace_size(q.dtype, B, H, Hkv, Tnew, S, d, start_pos, window)
     if workspace is None and need > 0:
         workspace = _torch().empty(need, dtype=_torch().uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if window:
+        st = _lib.load().attn_cached_local(_ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(out),
+                                           _ptr(lse), _dtype_code(q), B, H, Hkv, Tnew, S, S_cap, d,
+                                           int(start_pos), float(scale), int(window),
+                                           _ptr(workspace), ws_bytes,
+                                           _stream_handle(stream, q.device))
+        if st != _lib.OK:
+            raise AttnError(st, "attn_cached_local")
+        return out
     st = _lib.load().attn_cached(_ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(out), _ptr(lse),
                                  _dtype_code(q), B, H, Hkv, Tnew, S, S_cap, d, int(start_pos),
                                  float(scale), _ptr(workspace), ws_bytes,

@@ -22,7 +22,8 @@ KERNEL_NONE, KERNEL_SIMT, KERNEL_TCGEN05, KERNEL_SPLITKV = 0, 1, 2, 3
 KERNEL_NAMES = {KERNEL_NONE: "none", KERNEL_SIMT: "simt", KERNEL_TCGEN05: "tcgen05",
                 KERNEL_SPLITKV: "splitkv", -1: "rejected"}
 
-EXPORTS = ("attn_prefill", "attn_cached", "attn_cached_paged", "attn_cached_paged_workspace_size",
+EXPORTS = ("attn_prefill", "attn_cached", "attn_prefill_local", "attn_cached_local",
+           "attn_cached_local_workspace_size", "attn_cached_paged", "attn_cached_paged_workspace_size",
            "attn_kv_append_rope", "attn_cached_workspace_size", "attn_prefill_plan",
            "attn_cached_plan", "attn_status_string", "attn_device_status",
            "attn_set_wait_timeout_ns", "attn_test_set_flags", "attn_version")
@@ -68,6 +69,15 @@ def load() -> ctypes.CDLL:
             lib.attn_kv_append_rope.restype = c_int
             lib.attn_kv_append_rope.argtypes = [vp, vp, vp, vp, c_int, i64, i64, i64, i64, i64,
                                                 i64, f32, vp]
+            lib.attn_prefill_local.restype = c_int
+            lib.attn_prefill_local.argtypes = [vp, vp, vp, vp, vp, c_int, i64, i64, i64, i64, i64,
+                                               f32, i64, vp]
+            lib.attn_cached_local.restype = c_int
+            lib.attn_cached_local.argtypes = [vp, vp, vp, vp, vp, c_int, i64, i64, i64, i64, i64,
+                                              i64, i64, i64, f32, i64, vp, ctypes.c_size_t, vp]
+            lib.attn_cached_local_workspace_size.restype = ctypes.c_size_t
+            lib.attn_cached_local_workspace_size.argtypes = [c_int, i64, i64, i64, i64, i64, i64,
+                                                             i64, i64]
             lib.attn_cached_paged.restype = c_int
             lib.attn_cached_paged.argtypes = [vp, vp, vp, vp, vp, c_int, i64, i64, i64, i64, i64,
                                               vp, i64, i64, i64, vp, i64, f32, vp,

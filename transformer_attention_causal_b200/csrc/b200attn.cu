@@ -39,6 +39,7 @@ struct Problem {
     int64_t B, H, Hkv, Tq, S, S_cap, d, start_pos;
     int causal;
     bool cached;  // attn_cached: split-KV decode allowed
+    int64_t window = 0;  // local window (0: none); causal only
 };
 
 struct Plan {
@@ -46,7 +47,7 @@ struct Plan {
     // split-KV decode
     int R = 0, Rv = 0, nsplit = 1;
     bool wide = false;
-    int64_t chunk = 0, kv_end = 0;
+    int64_t chunk = 0, kv_end = 0, k_lo = 0;
     size_t ws_bytes = 0;
     // tcgen05 prefill
     int dch = 0, pair_mode = 0, n_qb = 0, units_per_level = 0, n_levels = 0;
@@ -58,7 +59,7 @@ bool empty_problem(const Problem& pb) { return pb.B == 0 || pb.H == 0 || pb.Tq =
 attn_status_t check_shape(const Problem& pb) {
     if (pb.dt != ATTN_F32 && pb.dt != ATTN_BF16 && pb.dt != ATTN_F16) return ATTN_ERR_INVALID_ARG;
     if (pb.B < 0 || pb.H < 0 || pb.Hkv < 0 || pb.Tq < 0 || pb.S < 0 || pb.S_cap < 0 ||
-        pb.d < 0 || pb.start_pos < 0)
+        pb.d < 0 || pb.start_pos < 0 || pb.window < 0 || (pb.window > 0 && !pb.causal))
         return ATTN_ERR_INVALID_ARG;
     if (empty_problem(pb)) return ATTN_OK;
     if (pb.Hkv == 0 || pb.H % pb.Hkv != 0 || pb.d == 0) return ATTN_ERR_INVALID_ARG;
@@ -92,7 +93,9 @@ void plan_decode(const Problem& pb, Plan& pl) {
     const int stage_keys = pl.wide ? 120 : 64;
     const int ctas_per_sm = pl.wide ? 1 : 2;
     pl.kv_end = std::min<int64_t>(pb.S, pb.start_pos + pb.Tq);
-    const int64_t tiles = (pl.kv_end + stage_keys - 1) / stage_keys;
+    // a local window: no row sees a key below the first row's window
+    pl.k_lo = pb.window > 0 ? std::max<int64_t>(0, pb.start_pos - pb.window + 1) : 0;
+    const int64_t tiles = (pl.kv_end - pl.k_lo + stage_keys - 1) / stage_keys;
     const int64_t units = pb.B * pb.Hkv;
     const int64_t slots = int64_t(kPlanSMs) * ctas_per_sm;
     // Pick the split count that fills the last wave of CTAs best; prefer fewer
@@ -218,6 +221,7 @@ attn_status_t run_simt(const Problem& pb, const void* q, const void* k, const vo
     sp.q = q; sp.k = k; sp.v = v; sp.o = o; sp.lse = lse;
     sp.B = pb.B; sp.H = pb.H; sp.Hkv = pb.Hkv; sp.Tq = pb.Tq; sp.S = pb.S; sp.S_cap = pb.S_cap;
     sp.d = pb.d; sp.start_pos = pb.start_pos; sp.scale = scale; sp.causal = pb.causal;
+    sp.window = pb.window;
     const int64_t rows = pb.B * pb.H * pb.Tq;
     const int64_t blocks = (rows + kSimtWarps - 1) / kSimtWarps;
     if (blocks > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
@@ -225,10 +229,10 @@ attn_status_t run_simt(const Problem& pb, const void* q, const void* k, const vo
     return launch_status();
 }
 
-template <typename T, int D, int R, bool PAGED>
+template <typename T, int D, int R, int MODE>
 attn_status_t launch_decode_RP(const DecodeParams& dp, cudaStream_t stream) {
     constexpr size_t smem = DecodeShape<D, R>::smem_bytes(sizeof(T));
-    auto kern = decode_splitkv_kernel<T, D, R, PAGED>;
+    auto kern = decode_splitkv_kernel<T, D, R, MODE>;
     static std::once_flag once[8];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -246,10 +250,10 @@ attn_status_t launch_decode_RP(const DecodeParams& dp, cudaStream_t stream) {
     return ATTN_OK;
 }
 
-template <typename T, int D, int R, bool PAGED>
+template <typename T, int D, int R, int MODE>
 attn_status_t launch_decode_wide_RP(const DecodeParams& dp, cudaStream_t stream) {
     constexpr size_t smem = WideShape<D, R>::smem_bytes(sizeof(T));
-    auto kern = decode_wide_kernel<T, D, R, PAGED>;
+    auto kern = decode_wide_kernel<T, D, R, MODE>;
     static std::once_flag once[8];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -269,14 +273,16 @@ attn_status_t launch_decode_wide_RP(const DecodeParams& dp, cudaStream_t stream)
 
 template <typename T, int D, int R>
 attn_status_t launch_decode_R(const DecodeParams& dp, cudaStream_t stream) {
-    return dp.paged ? launch_decode_RP<T, D, R, true>(dp, stream)
-                    : launch_decode_RP<T, D, R, false>(dp, stream);
+    if (dp.paged) return launch_decode_RP<T, D, R, kDecodePaged>(dp, stream);
+    if (dp.window > 0) return launch_decode_RP<T, D, R, kDecodeWindow>(dp, stream);
+    return launch_decode_RP<T, D, R, kDecodePlain>(dp, stream);
 }
 
 template <typename T, int D, int R>
 attn_status_t launch_decode_wide_R(const DecodeParams& dp, cudaStream_t stream) {
-    return dp.paged ? launch_decode_wide_RP<T, D, R, true>(dp, stream)
-                    : launch_decode_wide_RP<T, D, R, false>(dp, stream);
+    if (dp.paged) return launch_decode_wide_RP<T, D, R, kDecodePaged>(dp, stream);
+    if (dp.window > 0) return launch_decode_wide_RP<T, D, R, kDecodeWindow>(dp, stream);
+    return launch_decode_wide_RP<T, D, R, kDecodePlain>(dp, stream);
 }
 
 template <typename T, int D>
@@ -323,6 +329,7 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
     dp.G = int(pb.H / pb.Hkv); dp.Tnew = int(pb.Tq); dp.Rv = pl.Rv;
     dp.S = pb.S; dp.S_cap = pb.S_cap; dp.start_pos = pb.start_pos;
     dp.kv_end = pl.kv_end; dp.chunk = pl.chunk; dp.nsplit = pl.nsplit;
+    dp.k_lo = pl.k_lo; dp.window = pb.window;
     dp.scale_log2 = scale * 1.4426950408889634f;
     dp.timeout_ns = g_timeout_ns.load();
     dp.test_flags = g_test_flags.load();
@@ -342,6 +349,22 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
     }
 }
 
+template <typename T, int DCH, bool WINDOW>
+attn_status_t launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk,
+                                    const CUtensorMap& mv, const PrefillParams& pp, int64_t grid,
+                                    cudaStream_t stream) {
+    constexpr size_t smem = prefill_smem_bytes<DCH>();
+    auto kern = prefill_tcgen05_kernel<T, DCH, WINDOW>;
+    static std::once_flag once[8];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    attn_status_t st = ATTN_OK;
+    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
+    if (st != ATTN_OK) return st;
+    kern<<<unsigned(grid), kPfThreads, smem, stream>>>(mq, mk, mv, pp);
+    return launch_status();
+}
+
 template <typename T, int DCH>
 attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q, const void* k,
                                 const void* v, void* o, float* lse, float scale,
@@ -357,21 +380,14 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
     pp.B = int(pb.B); pp.H = int(pb.H); pp.Hkv = int(pb.Hkv); pp.G = int(pb.H / pb.Hkv);
     pp.Tq = int(pb.Tq); pp.S = pb.S; pp.start_pos = pb.start_pos; pp.d = int(pb.d);
     pp.causal = pb.causal; pp.pair_mode = pl.pair_mode; pp.n_qb = pl.n_qb;
+    pp.window = pb.window;
     pp.units_per_level = pl.units_per_level;
     pp.scale_log2 = scale * 1.4426950408889634f;
     pp.timeout_ns = g_timeout_ns.load();
     pp.test_flags = g_test_flags.load();
-    constexpr size_t smem = prefill_smem_bytes<DCH>();
-    auto kern = prefill_tcgen05_kernel<T, DCH>;
-    static std::once_flag once[8];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    attn_status_t st = ATTN_OK;
-    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
-    if (st != ATTN_OK) return st;
     const int64_t grid = int64_t(pl.units_per_level) * pl.n_levels;
-    kern<<<unsigned(grid), kPfThreads, smem, stream>>>(mq, mk, mv, pp);
-    return launch_status();
+    return pb.window > 0 ? launch_prefill_kernel<T, DCH, true>(mq, mk, mv, pp, grid, stream)
+                         : launch_prefill_kernel<T, DCH, false>(mq, mk, mv, pp, grid, stream);
 }
 
 template <typename T>
@@ -569,6 +585,48 @@ size_t attn_cached_paged_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H
     Plan pl;
     if (make_plan(paged_problem(dtype, B, H, Hkv, Tnew, d, max_kv_len), pl) != ATTN_OK) return 0;
     return pl.kernel == ATTN_KERNEL_SPLITKV ? pl.ws_bytes : 0;
+}
+
+attn_status_t attn_prefill_local(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t T,
+                                 int64_t d, float scale, int64_t window, void* stream) {
+    Problem pb{dtype, B, H, Hkv, T, T, T, d, 0, 1, false, window};
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    Plan pl;
+    attn_status_t st = make_plan(pb, pl);
+    if (st != ATTN_OK) return st;
+    st = check_pointers(pb, q, k, v, o, lse);
+    if (st != ATTN_OK) return st;
+    return dispatch(pb, pl, q, k, v, o, lse, scale, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_cached_local(const void* q, const void* k_hist, const void* v_hist, void* o,
+                                float* lse, attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                                int64_t Tnew, int64_t S, int64_t S_cap, int64_t d,
+                                int64_t start_pos, float scale, int64_t window, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    Problem pb{dtype, B, H, Hkv, Tnew, S, S_cap, d, start_pos, 1, true, window};
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    Plan pl;
+    attn_status_t st = make_plan(pb, pl);
+    if (st != ATTN_OK) return st;
+    st = check_pointers(pb, q, k_hist, v_hist, o, lse);
+    if (st != ATTN_OK) return st;
+    if (pl.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < pl.ws_bytes) return ATTN_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+    }
+    return dispatch(pb, pl, q, k_hist, v_hist, o, lse, scale, workspace,
+                    static_cast<cudaStream_t>(stream));
+}
+
+size_t attn_cached_local_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                                        int64_t Tnew, int64_t S, int64_t d, int64_t start_pos,
+                                        int64_t window) {
+    Problem pb{dtype, B, H, Hkv, Tnew, S, S, d, start_pos, 1, true, window};
+    Plan pl;
+    if (make_plan(pb, pl) != ATTN_OK) return 0;
+    return pl.ws_bytes;
 }
 
 size_t attn_cached_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,

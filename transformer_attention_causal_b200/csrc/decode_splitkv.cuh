@@ -42,6 +42,8 @@ struct DecodeParams {
     int B, H, Hkv, G, Tnew, Rv;  // Rv = G * Tnew valid rows per unit
     int64_t S, S_cap, start_pos;
     int64_t kv_end;      // min(S, start_pos + Tnew): last visible key + 1
+    int64_t k_lo;        // first key any row sees (0 without a local window)
+    int64_t window;      // local window w: row at p sees p - w < j <= p (0: none)
     int64_t chunk;       // keys per split (multiple of the stage size)
     int nsplit;
     float scale_log2;    // scale * log2(e)
@@ -182,9 +184,14 @@ struct DecodeShape {
     }
 };
 
-template <typename T, int D, int R, bool PAGED>
+// Kernel variants: contiguous cache, paged cache, local window.
+enum DecodeMode : int { kDecodePlain = 0, kDecodePaged = 1, kDecodeWindow = 2 };
+
+template <typename T, int D, int R, int MODE>
 __global__ void __launch_bounds__(160, 2)
 decode_splitkv_kernel(const DecodeParams p) {
+    constexpr bool PAGED = MODE == kDecodePaged;
+    constexpr bool WINDOW = MODE == kDecodeWindow;
     using Sh = DecodeShape<D, R>;
     constexpr int NW = Sh::NW, TK = Sh::TK, NST = Sh::NST, KW = Sh::KW, LPK = Sh::LPK,
                   KPG = Sh::KPG, CE = Sh::CE, NCH = Sh::NCH, GPW = Sh::GPW, LPR = Sh::LPR,
@@ -205,7 +212,7 @@ decode_splitkv_kernel(const DecodeParams p) {
     const int kvh = unit % p.Hkv;
     int64_t start_pos = p.start_pos, kv_end = p.kv_end;
     if constexpr (PAGED) decode_span(p, b, start_pos, kv_end);
-    const int64_t k_begin = int64_t(split) * p.chunk;
+    const int64_t k_begin = (WINDOW ? p.k_lo : 0) + int64_t(split) * p.chunk;
     const int64_t k_end = min64(kv_end, k_begin + p.chunk);
     const int nstages = k_end > k_begin ? int((k_end - k_begin + TK - 1) / TK) : 0;
 
@@ -281,6 +288,8 @@ decode_splitkv_kernel(const DecodeParams p) {
 #pragma unroll
     for (int r = 0; r < R; ++r)
         row_lim[r] = (r < p.Rv) ? start_pos + (r % p.Tnew) : -1;
+    // keys at or below row_lim[r] - wnd are outside a local window
+    const int64_t wnd = WINDOW ? p.window : (int64_t(1) << 62);
 
     float oacc[R][NCH][CE];
 #pragma unroll
@@ -355,7 +364,7 @@ decode_splitkv_kernel(const DecodeParams p) {
             bool vis = ki < nvalid;
 #pragma unroll
             for (int r = 0; r < R; ++r)
-                if (r == my_row) vis = vis && (j <= row_lim[r]);
+                if (r == my_row) vis = vis && (j <= row_lim[r]) && (!WINDOW || j > row_lim[r] - wnd);
             if (sub % (LPK / R) == 0) scw[kw * R + my_row] = vis ? acc[0] : -INFINITY;
         }
         __syncwarp();
@@ -627,9 +636,11 @@ __device__ __forceinline__ void load_elems(const T* src, float (&f)[N]) {
     }
 }
 
-template <typename T, int D, int R, bool PAGED>
+template <typename T, int D, int R, int MODE>
 __global__ void __launch_bounds__(512, 1)
 decode_wide_kernel(const DecodeParams p) {
+    constexpr bool PAGED = MODE == kDecodePaged;
+    constexpr bool WINDOW = MODE == kDecodeWindow;
     using Sh = WideShape<D, R>;
     constexpr int NW = Sh::NW, TK = Sh::TK, NST = Sh::NST, KW = Sh::KW, EA = Sh::EA, LPK = Sh::LPK,
                   KPG = Sh::KPG, GPW = Sh::GPW, EC = Sh::EC, LPR = Sh::LPR, SPL = Sh::SPL;
@@ -649,7 +660,7 @@ decode_wide_kernel(const DecodeParams p) {
     const int kvh = unit % p.Hkv;
     int64_t start_pos = p.start_pos, kv_end = p.kv_end;
     if constexpr (PAGED) decode_span(p, b, start_pos, kv_end);
-    const int64_t k_begin = int64_t(split) * p.chunk;
+    const int64_t k_begin = (WINDOW ? p.k_lo : 0) + int64_t(split) * p.chunk;
     const int64_t k_end = min64(kv_end, k_begin + p.chunk);
     const int nstages = k_end > k_begin ? int((k_end - k_begin + TK - 1) / TK) : 0;
 
@@ -721,7 +732,8 @@ decode_wide_kernel(const DecodeParams p) {
                           : make_float2(0.f, 0.f);
         }
     }
-    const bool single = p.Tnew == 1;  // every key below kv_end is visible
+    // one new token: every key in [k_lo, kv_end) is visible (window included)
+    const bool single = p.Tnew == 1;
     int64_t row_lim[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) row_lim[r] = (r < p.Rv) ? start_pos + (r % p.Tnew) : -1;
@@ -786,10 +798,11 @@ decode_wide_kernel(const DecodeParams p) {
             }
             bool vis = ki < nvalid;
             if (!single) {
+                const int64_t wnd = WINDOW ? p.window : (int64_t(1) << 62);
                 const int64_t j = k0 + ki;
 #pragma unroll
                 for (int r = 0; r < R; ++r)
-                    if (r == my_row) vis = vis && (j <= row_lim[r]);
+                    if (r == my_row) vis = vis && (j <= row_lim[r]) && (!WINDOW || j > row_lim[r] - wnd);
             }
             if (sub % (LPK / R) == 0) scw[kw * R + my_row] = vis ? acc[0] : -INFINITY;
         }

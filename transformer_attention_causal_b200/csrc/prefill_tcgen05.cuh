@@ -47,6 +47,7 @@ struct PrefillParams {
     int64_t start_pos;   // absolute position of query row 0
     int d;
     int causal;
+    int64_t window;      // local window w: the row at p sees p - w < j <= p (0: none)
     int pair_mode;       // 0: two heads share a row tile; 1: one head, two row tiles
     int n_qb;            // ceil(Tq / 128)
     int units_per_level;
@@ -94,6 +95,13 @@ __device__ __forceinline__ void mask_chunk(uint32_t (&r)[32], int last) {
 #pragma unroll
     for (int c = 0; c < 32; ++c)
         if (c > last) r[c] = 0xff800000u;  // -inf
+}
+
+// Columns before `first` of a 32-column chunk become -inf (a window's edge).
+__device__ __forceinline__ void mask_chunk_below(uint32_t (&r)[32], int first) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+        if (c < first) r[c] = 0xff800000u;  // -inf
 }
 
 // Maximum of a 32-column chunk (fp32 bits): four independent max3 chains.
@@ -151,17 +159,19 @@ constexpr size_t prefill_smem_bytes() {
     return 1024 + size_t(2 + PrefillRing<DCH>::NST) * DCH * kChunkBytes + 512;
 }
 
+// A slot's key tiles: it needs tiles [n_lo, n_kv); tiles in [n_full_lo,
+// n_full) are visible to every row of it, the others are masked.
 struct SlotInfo {
-    int h, q0, n_kv, n_full;
+    int h, q0, n_lo, n_kv, n_full_lo, n_full;
 };
 
+template <bool WINDOW>
 __device__ __forceinline__ SlotInfo prefill_slot(const PrefillParams& p, int h, int qb) {
     SlotInfo s;
     s.h = h;
     s.q0 = qb * 128;
     if (s.q0 >= p.Tq) {
-        s.n_kv = 0;
-        s.n_full = 0;
+        s.n_lo = s.n_kv = s.n_full_lo = s.n_full = 0;
         return s;
     }
     const int64_t qlast = min64(s.q0 + 127, p.Tq - 1);
@@ -169,6 +179,13 @@ __device__ __forceinline__ SlotInfo prefill_slot(const PrefillParams& p, int h, 
     s.n_kv = int((kv_end + 127) / 128);
     const int64_t full_c = p.causal ? (p.start_pos + s.q0 + 1) / 128 : (p.S / 128);
     s.n_full = int(min64(full_c, p.S / 128));
+    s.n_lo = s.n_full_lo = 0;
+    if (WINDOW) {
+        const int64_t first = max64(0, p.start_pos + s.q0 - p.window + 1);   // lowest key seen
+        const int64_t all_lo = max64(0, p.start_pos + qlast - p.window + 1);  // every row sees from here
+        s.n_lo = int(first / 128);
+        s.n_full_lo = int((all_lo + 127) / 128);
+    }
     return s;
 }
 
@@ -206,7 +223,7 @@ __device__ __forceinline__ void issue_PV(uint64_t dV0, uint32_t tmem, uint32_t i
                (accumulate || kk > 0) ? 1u : 0u);
 }
 
-template <typename T, int DCH>
+template <typename T, int DCH, bool WINDOW>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -244,18 +261,21 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int r2 = rem % (p.Hkv * half);
         kvh = r2 / half;
         const int h0 = kvh * p.G + 2 * (r2 % half);
-        slot[0] = prefill_slot(p, h0, qb);
-        slot[1] = prefill_slot(p, h0 + 1, qb);
+        slot[0] = prefill_slot<WINDOW>(p, h0, qb);
+        slot[1] = prefill_slot<WINDOW>(p, h0 + 1, qb);
     } else {
         const int n_levels = (p.n_qb + 1) / 2;
         const int qbp = n_levels - 1 - level;
         b = rem / p.H;
         const int h = rem % p.H;
         kvh = h / p.G;
-        slot[0] = prefill_slot(p, h, 2 * qbp);
-        slot[1] = prefill_slot(p, h, 2 * qbp + 1);
+        slot[0] = prefill_slot<WINDOW>(p, h, 2 * qbp);
+        slot[1] = prefill_slot<WINDOW>(p, h, 2 * qbp + 1);
     }
     const int nmax = max(slot[0].n_kv, slot[1].n_kv);
+    // first tile either slot needs (K/V loads start here)
+    const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
+                     : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&q_full[0]), 1);
@@ -264,6 +284,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(smem_u32(&kv_full[i]), 1);
             mbar_init(smem_u32(&kv_empty[i]), 1);
         }
+#pragma unroll
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_u32(&s_full[s]), 1);
             mbar_init(smem_u32(&p_ready[2 * s]), 4);      // one arrive per softmax warp
@@ -289,6 +310,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
+#pragma unroll
             for (int s = 0; s < 2; ++s) {
                 if (slot[s].n_kv == 0) continue;
                 const uint32_t bar = smem_u32(&q_full[s]);
@@ -299,7 +321,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             const int zkv = b * p.Hkv + kvh;
             int issued = 0;
-            const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * nmax;
+            const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * (nmax - nmin);
             for (int i = 0; i < n_loads; ++i) {
                 const int st = i % NST;
                 if (!mbar_wait(smem_u32(&kv_empty[st]), ((i / NST) & 1) ^ 1, p.timeout_ns, abort_flag))
@@ -309,12 +331,13 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 mbar_expect_tx(bar, DCH * kChunkBytes);
                 const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
                 for (int c = 0; c < DCH; ++c)
-                    tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64, (i >> 1) * 128,
+                    tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64, (nmin + (i >> 1)) * 128,
                                 zkv);
             }
             // no copy may still be landing in shared memory when the CTA exits
             for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
                 mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.timeout_ns, nullptr);
+#pragma unroll
             for (int s = 0; s < 2; ++s)
                 if (slot[s].n_kv > 0) mbar_wait(smem_u32(&q_full[s]), 0, p.timeout_ns, nullptr);
         }
@@ -328,20 +351,23 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             const uint64_t dK0 = smem_desc_sw128(sRing, 16, 1024);
             const uint64_t dV0 = smem_desc_sw128(sRing, kChunkBytes, 1024);
             bool ok = true;
+#pragma unroll
             for (int s = 0; s < 2 && ok; ++s)
                 if (slot[s].n_kv > 0) ok = mbar_wait(smem_u32(&q_full[s]), 0, p.timeout_ns, abort_flag);
             if (ok) ok = mbar_wait(smem_u32(&kv_full[0]), 0, p.timeout_ns, abort_flag);
             if (ok) {
                 tc_fence_after();
+#pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    if (slot[s].n_kv == 0) continue;
+                    if (slot[s].n_kv == 0 || slot[s].n_lo != nmin) continue;
                     issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, 0);
                     mma_commit(smem_u32(&s_full[s]));
                 }
                 mma_commit(smem_u32(&kv_empty[0]));
             }
-            for (int n = 0; n < nmax && ok; ++n) {
-                const int iV = 2 * n + 1, iK = 2 * n + 2;
+            // tile n of a slot is its (n - n_lo)-th: barrier phases count from there
+            for (int n = nmin; n < nmax && ok; ++n) {
+                const int iV = 2 * (n - nmin) + 1, iK = 2 * (n - nmin) + 2;
                 const int stV = iV % NST, stK = iK % NST;
                 const bool nextK = n + 1 < nmax;
                 ok = mbar_wait(smem_u32(&kv_full[stV]), (iV / NST) & 1, p.timeout_ns, abort_flag);
@@ -349,17 +375,25 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     ok = mbar_wait(smem_u32(&kv_full[stK]), (iK / NST) & 1, p.timeout_ns, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
+#pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    if (n >= slot[s].n_kv) continue;
+                    // a slot whose window starts at tile n + 1 only gets its first S here
+                    const bool first_next = WINDOW && n + 1 == slot[s].n_lo && n + 1 < slot[s].n_kv;
+                    if (first_next) {
+                        issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
+                        mma_commit(smem_u32(&s_full[s]));
+                    }
+                    if (n < slot[s].n_lo || n >= slot[s].n_kv) continue;
+                    const uint32_t par = uint32_t(n - slot[s].n_lo) & 1;
                     // P in two halves: the first 64 keys' MMAs start while the
                     // softmax is still producing the second half
-                    if (!mbar_wait(smem_u32(&p_ready[2 * s]), n & 1, p.timeout_ns, abort_flag)) {
+                    if (!mbar_wait(smem_u32(&p_ready[2 * s]), par, p.timeout_ns, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    issue_PV<0, DCH>(dV0, tmem, idO, s, stV, n > 0);
-                    if (!mbar_wait(smem_u32(&p_ready[2 * s + 1]), n & 1, p.timeout_ns, abort_flag)) {
+                    issue_PV<0, DCH>(dV0, tmem, idO, s, stV, n > slot[s].n_lo);
+                    if (!mbar_wait(smem_u32(&p_ready[2 * s + 1]), par, p.timeout_ns, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -393,8 +427,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             const float c2 = p.scale_log2;
             float m_run = -INFINITY, l = 0.f;
             bool ok = true;
-            for (int n = 0; n < sl.n_kv; ++n) {
-                ok = mbar_wait(smem_u32(&s_full[s]), n & 1, p.timeout_ns, abort_flag);
+            for (int n = sl.n_lo; n < sl.n_kv; ++n) {
+                ok = mbar_wait(smem_u32(&s_full[s]), uint32_t(n - sl.n_lo) & 1, p.timeout_ns, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
@@ -406,7 +440,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tmem_ld32(tS + 64, r2);
                 tmem_ld32(tS + 96, r3);
                 tmem_wait_ld();
-                const bool masked = n >= sl.n_full;
+                const bool masked = n >= sl.n_full || (WINDOW && n < sl.n_full_lo);
                 if (masked) {
                     int64_t lim = p.causal ? qpos - int64_t(n) * 128 : 127;
                     lim = min64(lim, p.S - 1 - int64_t(n) * 128);
@@ -415,10 +449,18 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     mask_chunk(r1, li - 32);
                     mask_chunk(r2, li - 64);
                     mask_chunk(r3, li - 96);
+                    if (WINDOW) {
+                        // keys at or below qpos - w are outside the window
+                        const int lo = int(max64(0, min64(128, qpos - p.window + 1 - int64_t(n) * 128)));
+                        mask_chunk_below(r0, lo);
+                        mask_chunk_below(r1, lo - 32);
+                        mask_chunk_below(r2, lo - 64);
+                        mask_chunk_below(r3, lo - 96);
+                    }
                 }
                 const float m_tile =
                     fmaxf(fmaxf(chunk_max(r0), chunk_max(r1)), fmaxf(chunk_max(r2), chunk_max(r3))) * c2;
-                if (n == 0) {
+                if (n == sl.n_lo) {
                     m_run = m_tile;
                 } else {
                     const bool need = m_tile - m_run > kRescaleThreshold;
@@ -444,7 +486,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 // stored at once; the first 64 keys are released to the MMA
                 // before the last 64 are computed.  r* then hold P in fp32.
                 const float2 c2v = make_float2(c2, c2);
-                const float2 negm = make_float2(-m_run, -m_run);
+                // a row that has seen no key yet (a window starting in a later
+                // tile) has m_run = -inf: its P must be 0, not NaN
+                const float m_use = WINDOW && m_run == -INFINITY ? 0.f : m_run;
+                const float2 negm = make_float2(-m_use, -m_use);
                 exp_chunk<T>(r0, c2v, negm, tS + 0);
                 exp_chunk<T>(r1, c2v, negm, tS + 16);
                 tmem_wait_st();

@@ -23,6 +23,7 @@ struct SimtParams {
     int64_t B, H, Hkv, Tq, S, S_cap, d, start_pos;
     float scale;
     int causal;
+    int64_t window;  // local window w: the row at p sees p - w < j <= p (0: none)
 };
 
 constexpr int kSimtWarps = 4;
@@ -52,6 +53,7 @@ simt_attention_kernel(const SimtParams p) {
 
     const int64_t pos = p.start_pos + i;
     const int64_t kv_end = p.causal ? min(p.S, pos + 1) : p.S;
+    const int64_t kv_lo = p.window > 0 ? max(int64_t(0), pos - p.window + 1) : int64_t(0);
 
     constexpr int kCols = kSimtMaxD / 32;
     float acc[kCols];
@@ -59,7 +61,7 @@ simt_attention_kernel(const SimtParams p) {
     for (int c = 0; c < kCols; ++c) acc[c] = 0.f;
     float m = -INFINITY, l = 0.f;
 
-    for (int64_t j0 = 0; j0 < kv_end; j0 += 32) {
+    for (int64_t j0 = kv_lo; j0 < kv_end; j0 += 32) {
         const int64_t j = j0 + lane;
         float s = -INFINITY;
         if (j < kv_end) {
