@@ -210,6 +210,20 @@ attn_status_t set_smem(K kernel, size_t bytes) {
                : ATTN_ERR_CUDA;
 }
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kPlanSMs;
+    int n = cached[dev].load();
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = kPlanSMs;
+        cached[dev].store(n);
+    }
+    return n;
+}
+
 attn_status_t launch_status() {
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -382,10 +396,13 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
     pp.causal = pb.causal; pp.pair_mode = pl.pair_mode; pp.n_qb = pl.n_qb;
     pp.window = pb.window;
     pp.units_per_level = pl.units_per_level;
+    pp.n_levels = pl.n_levels;
     pp.scale_log2 = scale * 1.4426950408889634f;
     pp.timeout_ns = g_timeout_ns.load();
     pp.test_flags = g_test_flags.load();
-    const int64_t grid = int64_t(pl.units_per_level) * pl.n_levels;
+    // persistent CTAs, one per SM (the kernel deals the units out itself)
+    const int64_t units = int64_t(pl.units_per_level) * pl.n_levels;
+    const int64_t grid = std::min<int64_t>(units, sm_count());
     return pb.window > 0 ? launch_prefill_kernel<T, DCH, true>(mq, mk, mv, pp, grid, stream)
                          : launch_prefill_kernel<T, DCH, false>(mq, mk, mv, pp, grid, stream);
 }

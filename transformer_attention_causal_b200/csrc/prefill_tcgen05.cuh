@@ -11,10 +11,14 @@
 //     every K/V tile loaded to shared memory feeds both heads ("Grouped-Query
 //     Attention" §5.1 without the repeat_interleave copy);
 //   * G odd (MHA, G = 1): one head, two consecutive 128-row tiles.
-// Units are launched heaviest first (longest causal row range first).
+// Units are ordered heaviest first (longest causal row range first) and dealt
+// to persistent CTAs (one per SM) in a snake order; barrier phases keep
+// counting across a CTA's units, so the next unit's Q and first K/V copies
+// and its first Q.K^T overlap the current unit's last tiles and epilogue.
 //
 // Warp roles (12 warps):
-//   warp 0      TMA producer: Q tiles once, then K_n, V_n into a ring of NST
+//   warp 0      TMA producer: per unit the Q tiles (once the previous unit's
+//               last Q.K^T has read them), then K_n, V_n into a ring of NST
 //               128-key stages (128-byte swizzle, zero fill past the end);
 //   warp 1      TMEM owner (allocates all 512 columns) and single-thread MMA
 //               issuer: S_s = Q_s K_n^T (SS MMA, M=N=128), O_s += P_s V_n
@@ -51,6 +55,7 @@ struct PrefillParams {
     int pair_mode;       // 0: two heads share a row tile; 1: one head, two row tiles
     int n_qb;            // ceil(Tq / 128)
     int units_per_level;
+    int n_levels;        // units = units_per_level * n_levels, heaviest level first
     float scale_log2;    // scale * log2(e)
     uint64_t timeout_ns;
     uint32_t test_flags;  // kTestSkipLoads: issue no K/V copies (timeout-path tests)
@@ -223,6 +228,39 @@ __device__ __forceinline__ void issue_PV(uint64_t dV0, uint32_t tmem, uint32_t i
                (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// The unit of work a CTA does at pass `unit`: its batch entry, K/V head and
+// two slots (heaviest first: the longest causal row range first).
+template <bool WINDOW>
+__device__ __forceinline__ void prefill_unit(const PrefillParams& p, int unit, int& b, int& kvh,
+                                             SlotInfo (&slot)[2]) {
+    const int level = unit / p.units_per_level;
+    const int rem = unit % p.units_per_level;
+    if (p.pair_mode == 0) {
+        const int half = p.G / 2;
+        const int qb = p.n_qb - 1 - level;
+        b = rem / (p.Hkv * half);
+        const int r2 = rem % (p.Hkv * half);
+        kvh = r2 / half;
+        const int h0 = kvh * p.G + 2 * (r2 % half);
+        slot[0] = prefill_slot<WINDOW>(p, h0, qb);
+        slot[1] = prefill_slot<WINDOW>(p, h0 + 1, qb);
+    } else {
+        const int qbp = p.n_levels - 1 - level;
+        b = rem / p.H;
+        const int h = rem % p.H;
+        kvh = h / p.G;
+        slot[0] = prefill_slot<WINDOW>(p, h, 2 * qbp);
+        slot[1] = prefill_slot<WINDOW>(p, h, 2 * qbp + 1);
+    }
+}
+
+// Unit dealt to this CTA at pass k: a snake over the grid (CTA c takes
+// units c, 2G - 1 - c, 2G + c, ...), so heavy and light units even out.
+__device__ __forceinline__ int prefill_pass_unit(int k) {
+    return (k & 1) == 0 ? k * int(gridDim.x) + int(blockIdx.x)
+                        : (k + 1) * int(gridDim.x) - 1 - int(blockIdx.x);
+}
+
 template <typename T, int DCH, bool WINDOW>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -237,7 +275,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t sRing = base + 2 * DCH * kChunkBytes;           // [NST][DCH] chunks
     uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + (2 + NST) * DCH * kChunkBytes);
     uint64_t* q_full = bars;            // 2
-    uint64_t* kv_full = bars + 2;       // NST
+    uint64_t* q_empty = bars + 2;       // 2
+    uint64_t* kv_full = bars + 4;       // NST
     uint64_t* kv_empty = kv_full + NST; // NST
     uint64_t* s_full = kv_empty + NST;  // 2
     uint64_t* p_ready = s_full + 2;     // [slot][half]: 4
@@ -248,48 +287,25 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int n_units = p.units_per_level * p.n_levels;
 
-    // ---- work unit (heaviest first)
-    const int level = blockIdx.x / p.units_per_level;
-    const int rem = blockIdx.x % p.units_per_level;
-    int b, kvh;
-    SlotInfo slot[2];
-    if (p.pair_mode == 0) {
-        const int half = p.G / 2;
-        const int qb = p.n_qb - 1 - level;
-        b = rem / (p.Hkv * half);
-        const int r2 = rem % (p.Hkv * half);
-        kvh = r2 / half;
-        const int h0 = kvh * p.G + 2 * (r2 % half);
-        slot[0] = prefill_slot<WINDOW>(p, h0, qb);
-        slot[1] = prefill_slot<WINDOW>(p, h0 + 1, qb);
-    } else {
-        const int n_levels = (p.n_qb + 1) / 2;
-        const int qbp = n_levels - 1 - level;
-        b = rem / p.H;
-        const int h = rem % p.H;
-        kvh = h / p.G;
-        slot[0] = prefill_slot<WINDOW>(p, h, 2 * qbp);
-        slot[1] = prefill_slot<WINDOW>(p, h, 2 * qbp + 1);
-    }
-    const int nmax = max(slot[0].n_kv, slot[1].n_kv);
-    // first tile either slot needs (K/V loads start here)
-    const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
-                     : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
-
+    // Persistent CTAs work through their units as one pipeline: every barrier
+    // keeps counting phases across units (each role tracks its own counts),
+    // so the producer loads the next unit's Q and first K/V tiles while this
+    // unit's last tiles and epilogue run, and the issuer starts the next
+    // unit's first Q.K^T as soon as they land.
     if (threadIdx.x == 0) {
-        mbar_init(smem_u32(&q_full[0]), 1);
-        mbar_init(smem_u32(&q_full[1]), 1);
-        for (int i = 0; i < NST; ++i) {
-            mbar_init(smem_u32(&kv_full[i]), 1);
-            mbar_init(smem_u32(&kv_empty[i]), 1);
-        }
-#pragma unroll
         for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&q_full[s]), 1);
+            mbar_init(smem_u32(&q_empty[s]), 1);
             mbar_init(smem_u32(&s_full[s]), 1);
             mbar_init(smem_u32(&p_ready[2 * s]), 4);      // one arrive per softmax warp
             mbar_init(smem_u32(&p_ready[2 * s + 1]), 4);
             mbar_init(smem_u32(&o_done[s]), 1);
+        }
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(smem_u32(&kv_full[i]), 1);
+            mbar_init(smem_u32(&kv_empty[i]), 1);
         }
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
@@ -310,36 +326,57 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
+            uint32_t qcount[2] = {0, 0};   // Q loads per slot so far
+            int64_t li = 0;                // K/V loads so far (ring position)
+            bool ok = true;
+            for (int pass = 0; ok; ++pass) {
+                const int unit = prefill_pass_unit(pass);
+                if (unit >= n_units) break;
+                int b, kvh;
+                SlotInfo slot[2];
+                prefill_unit<WINDOW>(p, unit, b, kvh, slot);
+                const int nmax = max(slot[0].n_kv, slot[1].n_kv);
+                const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
+                                 : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
 #pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                if (slot[s].n_kv == 0) continue;
-                const uint32_t bar = smem_u32(&q_full[s]);
-                mbar_expect_tx(bar, DCH * kChunkBytes);
-                for (int c = 0; c < DCH; ++c)
-                    tma_load_3d(sQ + (s * DCH + c) * kChunkBytes, &tmQ, bar, c * 64, slot[s].q0,
-                                b * p.H + slot[s].h);
-            }
-            const int zkv = b * p.Hkv + kvh;
-            int issued = 0;
-            const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * (nmax - nmin);
-            for (int i = 0; i < n_loads; ++i) {
-                const int st = i % NST;
-                if (!mbar_wait(smem_u32(&kv_empty[st]), ((i / NST) & 1) ^ 1, p.timeout_ns, abort_flag))
-                    break;
-                issued = i + 1;
-                const uint32_t bar = smem_u32(&kv_full[st]);
-                mbar_expect_tx(bar, DCH * kChunkBytes);
-                const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
-                for (int c = 0; c < DCH; ++c)
-                    tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64, (nmin + (i >> 1)) * 128,
-                                zkv);
+                for (int s = 0; s < 2; ++s) {
+                    if (slot[s].n_kv == 0) continue;
+                    // the previous unit's Q.K^T MMAs of this slot are done with Q
+                    if (qcount[s] > 0 &&
+                        !mbar_wait(smem_u32(&q_empty[s]), (qcount[s] - 1) & 1, p.timeout_ns, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = smem_u32(&q_full[s]);
+                    mbar_expect_tx(bar, DCH * kChunkBytes);
+                    for (int c = 0; c < DCH; ++c)
+                        tma_load_3d(sQ + (s * DCH + c) * kChunkBytes, &tmQ, bar, c * 64, slot[s].q0,
+                                    b * p.H + slot[s].h);
+                    ++qcount[s];
+                }
+                const int zkv = b * p.Hkv + kvh;
+                const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * (nmax - nmin);
+                for (int i = 0; i < n_loads && ok; ++i, ++li) {
+                    const int st = int(li % NST);
+                    if (!mbar_wait(smem_u32(&kv_empty[st]), uint32_t((li / NST) & 1) ^ 1, p.timeout_ns,
+                                   abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = smem_u32(&kv_full[st]);
+                    mbar_expect_tx(bar, DCH * kChunkBytes);
+                    const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+                    for (int c = 0; c < DCH; ++c)
+                        tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64,
+                                    (nmin + (i >> 1)) * 128, zkv);
+                }
             }
             // no copy may still be landing in shared memory when the CTA exits
-            for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
-                mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.timeout_ns, nullptr);
-#pragma unroll
+            for (int64_t i = li - 1; i >= 0 && i >= li - NST; --i)
+                mbar_wait(smem_u32(&kv_full[i % NST]), uint32_t((i / NST) & 1), p.timeout_ns, nullptr);
             for (int s = 0; s < 2; ++s)
-                if (slot[s].n_kv > 0) mbar_wait(smem_u32(&q_full[s]), 0, p.timeout_ns, nullptr);
+                if (qcount[s] > 0)
+                    mbar_wait(smem_u32(&q_full[s]), (qcount[s] - 1) & 1, p.timeout_ns, nullptr);
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
@@ -350,64 +387,92 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
             const uint64_t dK0 = smem_desc_sw128(sRing, 16, 1024);
             const uint64_t dV0 = smem_desc_sw128(sRing, kChunkBytes, 1024);
+            uint32_t qcount[2] = {0, 0};   // units started per slot
+            uint32_t pcount[2] = {0, 0};   // tiles whose P was consumed, per slot
+            int64_t li = 0;                // K/V loads consumed (ring position)
             bool ok = true;
-#pragma unroll
-            for (int s = 0; s < 2 && ok; ++s)
-                if (slot[s].n_kv > 0) ok = mbar_wait(smem_u32(&q_full[s]), 0, p.timeout_ns, abort_flag);
-            if (ok) ok = mbar_wait(smem_u32(&kv_full[0]), 0, p.timeout_ns, abort_flag);
-            if (ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    if (slot[s].n_kv == 0 || slot[s].n_lo != nmin) continue;
-                    issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, 0);
-                    mma_commit(smem_u32(&s_full[s]));
-                }
-                mma_commit(smem_u32(&kv_empty[0]));
-            }
-            // tile n of a slot is its (n - n_lo)-th: barrier phases count from there
-            for (int n = nmin; n < nmax && ok; ++n) {
-                const int iV = 2 * (n - nmin) + 1, iK = 2 * (n - nmin) + 2;
-                const int stV = iV % NST, stK = iK % NST;
-                const bool nextK = n + 1 < nmax;
-                ok = mbar_wait(smem_u32(&kv_full[stV]), (iV / NST) & 1, p.timeout_ns, abort_flag);
-                if (ok && nextK)
-                    ok = mbar_wait(smem_u32(&kv_full[stK]), (iK / NST) & 1, p.timeout_ns, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
+            for (int pass = 0; ok; ++pass) {
+                const int unit = prefill_pass_unit(pass);
+                if (unit >= n_units) break;
+                int b, kvh;
+                SlotInfo slot[2];
+                prefill_unit<WINDOW>(p, unit, b, kvh, slot);
+                const int nmax = max(slot[0].n_kv, slot[1].n_kv);
+                const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
+                                 : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    // a slot whose window starts at tile n + 1 only gets its first S here
-                    const bool first_next = WINDOW && n + 1 == slot[s].n_lo && n + 1 < slot[s].n_kv;
-                    if (first_next) {
+                    if (slot[s].n_kv == 0 || !ok) continue;
+                    ok = mbar_wait(smem_u32(&q_full[s]), qcount[s] & 1, p.timeout_ns, abort_flag);
+                    ++qcount[s];
+                }
+                if (ok) ok = mbar_wait(smem_u32(&kv_full[li % NST]), uint32_t((li / NST) & 1), p.timeout_ns,
+                                       abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                {
+                    const int stK = int(li % NST);
+#pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        if (slot[s].n_kv == 0 || slot[s].n_lo != nmin) continue;
                         issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
                         mma_commit(smem_u32(&s_full[s]));
+                        if (nmin + 1 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
                     }
-                    if (n < slot[s].n_lo || n >= slot[s].n_kv) continue;
-                    const uint32_t par = uint32_t(n - slot[s].n_lo) & 1;
-                    // P in two halves: the first 64 keys' MMAs start while the
-                    // softmax is still producing the second half
-                    if (!mbar_wait(smem_u32(&p_ready[2 * s]), par, p.timeout_ns, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+                    mma_commit(smem_u32(&kv_empty[stK]));
+                    ++li;
+                }
+                for (int n = nmin; n < nmax && ok; ++n) {
+                    const int64_t iV = li, iK = li + 1;
+                    const int stV = int(iV % NST), stK = int(iK % NST);
+                    const bool nextK = n + 1 < nmax;
+                    ok = mbar_wait(smem_u32(&kv_full[stV]), uint32_t((iV / NST) & 1), p.timeout_ns, abort_flag);
+                    if (ok && nextK)
+                        ok = mbar_wait(smem_u32(&kv_full[stK]), uint32_t((iK / NST) & 1), p.timeout_ns,
+                                       abort_flag);
+                    if (!ok) break;
                     tc_fence_after();
-                    issue_PV<0, DCH>(dV0, tmem, idO, s, stV, n > slot[s].n_lo);
-                    if (!mbar_wait(smem_u32(&p_ready[2 * s + 1]), par, p.timeout_ns, abort_flag)) {
-                        ok = false;
-                        break;
+#pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        // a slot whose window starts at tile n + 1 only gets its first S here
+                        const bool first_next = WINDOW && n + 1 == slot[s].n_lo && n + 1 < slot[s].n_kv;
+                        if (first_next) {
+                            issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
+                            mma_commit(smem_u32(&s_full[s]));
+                            if (n + 2 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
+                        }
+                        if (!ok || n < slot[s].n_lo || n >= slot[s].n_kv) continue;
+                        const uint32_t par = pcount[s] & 1;
+                        // P in two halves: the first 64 keys' MMAs start while the
+                        // softmax is still producing the second half
+                        if (!mbar_wait(smem_u32(&p_ready[2 * s]), par, p.timeout_ns, abort_flag)) {
+                            ok = false;
+                            continue;
+                        }
+                        tc_fence_after();
+                        issue_PV<0, DCH>(dV0, tmem, idO, s, stV, n > slot[s].n_lo);
+                        if (!mbar_wait(smem_u32(&p_ready[2 * s + 1]), par, p.timeout_ns, abort_flag)) {
+                            ok = false;
+                            continue;
+                        }
+                        tc_fence_after();
+                        issue_PV<4, DCH>(dV0, tmem, idO, s, stV, true);
+                        ++pcount[s];
+                        if (n == slot[s].n_kv - 1) mma_commit(smem_u32(&o_done[s]));
+                        if (n + 1 < slot[s].n_kv) {
+                            issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
+                            mma_commit(smem_u32(&s_full[s]));
+                            if (n + 2 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
+                        }
                     }
-                    tc_fence_after();
-                    issue_PV<4, DCH>(dV0, tmem, idO, s, stV, true);
-                    if (n == slot[s].n_kv - 1) mma_commit(smem_u32(&o_done[s]));
-                    if (n + 1 < slot[s].n_kv) {
-                        issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
-                        mma_commit(smem_u32(&s_full[s]));
+                    if (!ok) break;
+                    mma_commit(smem_u32(&kv_empty[stV]));
+                    ++li;
+                    if (nextK) {
+                        mma_commit(smem_u32(&kv_empty[stK]));
+                        ++li;
                     }
                 }
-                if (!ok) break;
-                mma_commit(smem_u32(&kv_empty[stV]));
-                if (nextK) mma_commit(smem_u32(&kv_empty[stK]));
             }
             // every MMA issued must finish before TMEM is released
             mma_commit(smem_u32(drain));
@@ -419,17 +484,25 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int s = (warp - 4) >> 2;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
-        const SlotInfo sl = slot[s];
-        if (sl.n_kv > 0) {
-            const uint32_t tS = tmem + (uint32_t(wq * 32) << 16) + s * 128;
-            const uint32_t tO = tmem + (uint32_t(wq * 32) << 16) + 256 + s * 128;
+        const uint32_t tS = tmem + (uint32_t(wq * 32) << 16) + s * 128;
+        const uint32_t tO = tmem + (uint32_t(wq * 32) << 16) + 256 + s * 128;
+        const float c2 = p.scale_log2;
+        uint32_t scount = 0, ocount = 0;   // S tiles and units consumed by this slot
+        bool ok = true;
+        for (int pass = 0; ok; ++pass) {
+            const int unit = prefill_pass_unit(pass);
+            if (unit >= n_units) break;
+            int b, kvh;
+            SlotInfo slot[2];
+            prefill_unit<WINDOW>(p, unit, b, kvh, slot);
+            const SlotInfo sl = slot[s];
+            if (sl.n_kv == 0) continue;
             const int64_t qpos = p.start_pos + sl.q0 + row;
-            const float c2 = p.scale_log2;
             float m_run = -INFINITY, l = 0.f;
-            bool ok = true;
             for (int n = sl.n_lo; n < sl.n_kv; ++n) {
-                ok = mbar_wait(smem_u32(&s_full[s]), uint32_t(n - sl.n_lo) & 1, p.timeout_ns, abort_flag);
+                ok = mbar_wait(smem_u32(&s_full[s]), scount & 1, p.timeout_ns, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
+                ++scount;
                 if (!ok) break;
                 tc_fence_after();
                 // All 128 scores of this row in registers (one wait: TMEM
@@ -506,7 +579,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 l += chunk_sum(r0) + chunk_sum(r1) + chunk_sum(r2) + chunk_sum(r3);
             }
             // ---- epilogue: O / l, rounded to the output type
-            if (ok) ok = mbar_wait(smem_u32(&o_done[s]), 0, p.timeout_ns, abort_flag);
+            if (ok) ok = mbar_wait(smem_u32(&o_done[s]), ocount & 1, p.timeout_ns, abort_flag);
+            ++ocount;
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 tc_fence_after();
