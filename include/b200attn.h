@@ -232,6 +232,39 @@ ATTN_API size_t attn_cached_paged_workspace_size(attn_dtype_t dtype, int64_t B, 
                                                  int64_t Hkv, int64_t Tnew, int64_t d,
                                                  int64_t max_kv_len);
 
+/*
+ * Backward pass of full-sequence attention ("Causal Multi-Head Self-Attention",
+ * Two exact full-sequence algorithms: the memory-linear path keeps only each
+ * row's statistics from the forward and rebuilds every probability from Q, K
+ * and them; a context upstream yields query, key and value gradients through
+ * the exact softmax vector-Jacobian product; Causal mask: a masked score
+ * carries exactly zero gradient).
+ *   q [B,H,T,d], k/v [B,Hkv,T,d]: the forward's inputs; o [B,H,T,d]: its
+ *   output; lse [B,H,T] float32: the row statistic (natural log) that
+ *   attn_prefill wrote for the same q, k, v, scale and causal; dout
+ *   [B,H,T,d]: the gradient of the loss with respect to o.
+ *   dq [B,H,T,d], dk/dv [B,Hkv,T,d]: overwritten with the gradients; dk and dv
+ *   hold the sums over the G = H/Hkv query heads that share each K/V head.
+ *   Every tensor row-major and contiguous, 16-byte aligned, one dtype (bf16 or
+ *   f16) for all but lse.
+ *   workspace: at least attn_prefill_backward_workspace_size() bytes, 16-byte
+ *   aligned; contents on entry irrelevant, scratch afterwards.
+ * Supported: bf16/f16 with d a multiple of 16 in [64, 128] (the tensor-core
+ * kernels); float32 and other head widths return ATTN_ERR_UNSUPPORTED.
+ * Errors as for attn_prefill plus ATTN_ERR_WORKSPACE; checks precede every
+ * launch.  An empty problem launches nothing (with H = 0 but B*Hkv*T > 0,
+ * dk and dv are set to zero).  Three kernels on `stream`, no allocation, no
+ * synchronisation.
+ */
+ATTN_API size_t attn_prefill_backward_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H,
+                                                     int64_t Hkv, int64_t T, int64_t d);
+ATTN_API attn_status_t attn_prefill_backward(const void* q, const void* k, const void* v,
+                                             const void* o, const float* lse, const void* dout,
+                                             void* dq, void* dk, void* dv, attn_dtype_t dtype,
+                                             int64_t B, int64_t H, int64_t Hkv, int64_t T,
+                                             int64_t d, float scale, int causal, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+
 /* Bytes of workspace attn_cached needs for this problem (0 if none).  Pure
  * host arithmetic; valid without a GPU.  Returns 0 for arguments that
  * attn_cached would reject. */

@@ -205,3 +205,41 @@ def test_paged_limits(lib):
     assert paged(lib, B=64, H=32, Hkv=8, max_pages=128, num_pages=8192, page_size=64,
                  max_kv_len=8192) == WORKSPACE
     assert lib.attn_cached_paged_workspace_size(F32, 64, 32, 8, 1, 128, 8192) == 0
+
+
+def backward(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+             dt=BF16, B=1, H=4, Hkv=2, T=300, d=128, scale=0.125, causal=1, ws=FAKE,
+             ws_bytes=1 << 20):
+    return lib.attn_prefill_backward(q, k, v, o, lse, do, dq, dk, dv, dt, B, H, Hkv, T, d, scale,
+                                     causal, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kwargs", [
+    dict(q=None), dict(k=None), dict(v=None), dict(o=None), dict(lse=None), dict(do=None),
+    dict(dq=None), dict(dk=None), dict(dv=None), dict(dq=MISALIGNED), dict(do=MISALIGNED),
+    dict(lse=ctypes.c_void_p(0x10002)), dict(ws=MISALIGNED),
+    dict(B=-1), dict(T=-1), dict(Hkv=0), dict(H=6, Hkv=4), dict(dt=7), dict(scale=float("nan")),
+])
+def test_backward_rejects_invalid_arguments(lib, kwargs):
+    assert backward(lib, **kwargs) == INVALID
+
+
+@pytest.mark.parametrize("kwargs", [dict(dt=F32), dict(d=48), dict(d=136), dict(d=72)])
+def test_backward_rejects_unsupported_shapes(lib, kwargs):
+    assert backward(lib, **kwargs) == UNSUPPORTED
+
+
+def test_backward_workspace(lib):
+    # two float32 row statistics per padded query row: 300 rows pad to 384
+    need = lib.attn_prefill_backward_workspace_size(BF16, 2, 4, 2, 300, 128)
+    assert need == 2 * 2 * 4 * 384 * 4
+    assert lib.attn_prefill_backward_workspace_size(F32, 2, 4, 2, 300, 128) == 0
+    assert lib.attn_prefill_backward_workspace_size(BF16, 2, 4, 2, 0, 128) == 0
+    assert backward(lib, B=2, ws=FAKE, ws_bytes=need - 1) == WORKSPACE
+    assert backward(lib, B=2, ws=None, ws_bytes=need) == WORKSPACE
+
+
+def test_backward_empty_problem(lib):
+    # T = 0: nothing to do, null pointers allowed
+    assert backward(lib, q=None, k=None, v=None, o=None, lse=None, do=None, dq=None, dk=None,
+                    dv=None, ws=None, ws_bytes=0, T=0) == 0

@@ -16,7 +16,8 @@ import ctypes
 from . import _lib
 from ._lib import AttnError
 
-__all__ = ["prefill", "cached", "cached_paged", "kv_append_rope", "cached_workspace_size",
+__all__ = ["prefill", "prefill_backward", "cached", "cached_paged", "kv_append_rope",
+           "cached_workspace_size", "prefill_backward_workspace_size",
            "cached_paged_workspace_size", "prefill_plan", "cached_plan", "device_status",
            "set_wait_timeout_ns", "AttnError"]
 
@@ -91,6 +92,43 @@ def prefill(q, k, v, *, scale: float, causal: bool = True, out=None, lse=None, s
     if st != _lib.OK:
         raise AttnError(st, "attn_prefill")
     return out
+
+
+def prefill_backward_workspace_size(dtype, B, H, Hkv, T, d) -> int:
+    return int(_lib.load().attn_prefill_backward_workspace_size(_code_of(dtype), B, H, Hkv, T, d))
+
+
+def prefill_backward(q, k, v, out, lse, dout, *, scale: float, causal: bool = True, dq=None,
+                     dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of full-sequence attention.  q, out, dout [B,H,T,d]; k, v
+    [B,Hkv,T,d]; lse float32 [B,H,T] as written by ``prefill`` for the same
+    inputs.  Returns (dq, dk, dv); dk and dv are summed over the query heads
+    that share each K/V head."""
+    torch = _torch()
+    _check(q, k, v, out, lse, dout, dq, dk, dv, workspace)
+    B, H, T, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (B, Hkv, T, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, Hkv, T, d] matching q")
+    if tuple(out.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("out and dout must match q")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T):
+        raise ValueError("lse must be float32 [B, H, T]")
+    dq = q.new_empty(q.shape) if dq is None else dq
+    dk = k.new_empty(k.shape) if dk is None else dk
+    dv = v.new_empty(v.shape) if dv is None else dv
+    need = prefill_backward_workspace_size(q.dtype, B, H, Hkv, T, d)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.load().attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                           _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                           _dtype_code(q), B, H, Hkv, T, d, float(scale),
+                                           int(bool(causal)), _ptr(workspace), ws_bytes,
+                                           _stream_handle(stream, q.device))
+    if st != _lib.OK:
+        raise AttnError(st, "attn_prefill_backward")
+    return dq, dk, dv
 
 
 def cached_workspace_size(dtype, B, H, Hkv, Tnew, S, d, start_pos, window: int = 0) -> int:

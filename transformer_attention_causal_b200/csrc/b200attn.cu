@@ -14,6 +14,7 @@
 #include "b200attn.h"
 #include "decode_splitkv.cuh"
 #include "kv_append.cuh"
+#include "prefill_backward.cuh"
 #include "prefill_tcgen05.cuh"
 #include "simt_attn.cuh"
 
@@ -476,6 +477,69 @@ attn_status_t launch_append(AppendParams& ap, cudaStream_t stream) {
 
 }  // namespace
 
+namespace {
+
+// Shapes the tensor-core backward kernels take.
+attn_status_t check_backward(const Problem& pb) {
+    attn_status_t st = check_shape(pb);
+    if (st != ATTN_OK || empty_problem(pb)) return st;
+    if (pb.dt == ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+    if (pb.d % 16 != 0 || pb.d < 64 || pb.d > 128) return ATTN_ERR_UNSUPPORTED;
+    const int64_t n_t = (pb.Tq + 127) / 128;
+    if (n_t * pb.B * pb.H >= (int64_t(1) << 31) || pb.Tq >= (int64_t(1) << 30) ||
+        pb.S_cap * pb.d * 2 >= (int64_t(1) << 40))
+        return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+size_t backward_ws_bytes(const Problem& pb) {
+    const int64_t tpad = (pb.Tq + 127) / 128 * 128;
+    const size_t bytes = size_t(2) * size_t(pb.B * pb.H * tpad) * sizeof(float);
+    return (bytes + 255) & ~size_t(255);
+}
+
+template <typename K>
+attn_status_t set_smem_once(K kern, size_t bytes, std::once_flag (&once)[8]) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    attn_status_t st = ATTN_OK;
+    std::call_once(once[dev & 7], [&] { st = set_smem(kern, bytes); });
+    return st;
+}
+
+template <typename T, int DCH>
+attn_status_t launch_backward(const Problem& pb, BwdParams& bp, const void* q, const void* k,
+                              const void* v, const void* dout, cudaStream_t stream) {
+    if (get_encoder() != ATTN_OK) return ATTN_ERR_CUDA;
+    CUtensorMap mq, mk, mv, mdo;
+    if (encode_rows(&mq, q, pb.dt, pb.d, pb.Tq, pb.Tq, pb.B * pb.H) != ATTN_OK ||
+        encode_rows(&mdo, dout, pb.dt, pb.d, pb.Tq, pb.Tq, pb.B * pb.H) != ATTN_OK ||
+        encode_rows(&mk, k, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK ||
+        encode_rows(&mv, v, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK)
+        return ATTN_ERR_CUDA;
+    const int64_t rows = int64_t(bp.B) * bp.H * bp.Tpad;
+    const int64_t pre_blocks = std::min<int64_t>((rows + 15) / 16, int64_t(sm_count()) * 16);
+    bwd_preprocess_kernel<T><<<unsigned(pre_blocks), 256, 0, stream>>>(bp);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
+
+    static std::once_flag once_kv[8], once_q[8];
+    constexpr size_t smem_kv = bwd_dkdv_smem_bytes<DCH>();
+    constexpr size_t smem_q = bwd_dq_smem_bytes<DCH>();
+    auto kern_kv = bwd_dkdv_kernel<T, DCH>;
+    auto kern_q = bwd_dq_kernel<T, DCH>;
+    if (set_smem_once(kern_kv, smem_kv, once_kv) != ATTN_OK ||
+        set_smem_once(kern_q, smem_q, once_q) != ATTN_OK)
+        return ATTN_ERR_CUDA;
+    kern_kv<<<unsigned(int64_t(bp.n_t) * bp.B * bp.Hkv), kBwdThreads, smem_kv, stream>>>(mq, mk, mv,
+                                                                                        mdo, bp);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
+    kern_q<<<unsigned(int64_t(bp.n_t) * bp.B * bp.H), kBwdThreads, smem_q, stream>>>(mq, mk, mv, mdo,
+                                                                                    bp);
+    return launch_status();
+}
+
+}  // namespace
+
 extern "C" {
 
 attn_status_t attn_kv_append_rope(const void* k_new, const void* v_new, void* k_cache,
@@ -520,6 +584,60 @@ attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o,
     st = check_pointers(pb, q, k, v, o, lse);
     if (st != ATTN_OK) return st;
     return dispatch(pb, pl, q, k, v, o, lse, scale, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+size_t attn_prefill_backward_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
+                                            int64_t T, int64_t d) {
+    Problem pb{dtype, B, H, Hkv, T, T, T, d, 0, 1, false};
+    if (check_backward(pb) != ATTN_OK || empty_problem(pb)) return 0;
+    return backward_ws_bytes(pb);
+}
+
+attn_status_t attn_prefill_backward(const void* q, const void* k, const void* v, const void* o,
+                                    const float* lse, const void* dout, void* dq, void* dk,
+                                    void* dv, attn_dtype_t dtype, int64_t B, int64_t H,
+                                    int64_t Hkv, int64_t T, int64_t d, float scale, int causal,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    Problem pb{dtype, B, H, Hkv, T, T, T, d, 0, causal ? 1 : 0, false};
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    attn_status_t st = check_backward(pb);
+    if (st != ATTN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (empty_problem(pb)) {
+        // no query head reads the keys: their gradients are zero
+        const size_t kv_bytes = size_t(B * Hkv * T * d) * esize(dtype);
+        if (kv_bytes == 0) return ATTN_OK;
+        if (!dk || !dv) return ATTN_ERR_INVALID_ARG;
+        return cudaMemsetAsync(dk, 0, kv_bytes, s) == cudaSuccess &&
+                       cudaMemsetAsync(dv, 0, kv_bytes, s) == cudaSuccess
+                   ? ATTN_OK
+                   : ATTN_ERR_CUDA;
+    }
+    const void* bufs[8] = {q, k, v, o, dout, dq, dk, dv};
+    for (const void* ptr : bufs)
+        if (!ptr || !aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+    if (!lse || !aligned4(lse)) return ATTN_ERR_INVALID_ARG;
+    const size_t need = backward_ws_bytes(pb);
+    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+    BwdParams bp;
+    bp.o = o; bp.dout = dout; bp.lse = lse;
+    bp.dq = dq; bp.dk = dk; bp.dv = dv;
+    bp.B = int(B); bp.H = int(H); bp.Hkv = int(Hkv); bp.G = int(H / Hkv); bp.T = int(T);
+    bp.n_t = int((T + 127) / 128);
+    bp.Tpad = bp.n_t * 128;
+    bp.d = int(d); bp.causal = causal ? 1 : 0;
+    bp.nl = static_cast<float*>(workspace);
+    bp.dd = bp.nl + size_t(B * H) * bp.Tpad;
+    bp.scale = scale;
+    bp.scale_log2 = scale * 1.4426950408889634f;
+    bp.timeout_ns = g_timeout_ns.load();
+    const bool bf16 = dtype == ATTN_BF16;
+    if (d <= 64)
+        return bf16 ? launch_backward<__nv_bfloat16, 1>(pb, bp, q, k, v, dout, s)
+                    : launch_backward<__half, 1>(pb, bp, q, k, v, dout, s);
+    return bf16 ? launch_backward<__nv_bfloat16, 2>(pb, bp, q, k, v, dout, s)
+                : launch_backward<__half, 2>(pb, bp, q, k, v, dout, s);
 }
 
 attn_status_t attn_cached(const void* q, const void* k_hist, const void* v_hist, void* o,

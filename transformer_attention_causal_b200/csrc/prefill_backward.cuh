@@ -1,0 +1,664 @@
+// Backward pass of full-sequence attention on the 5th-generation tensor cores.
+//
+// The forward saves one statistic per query row, lse = m + ln(l) (the row
+// maximum and exponential sum folded into one number), and the backward
+// rebuilds every probability it needs from Q, K and that statistic, so no
+// T x T matrix is ever stored ("Causal Multi-Head Self-Attention", Two exact
+// full-sequence algorithms: the Flash path keeps only the row statistics and
+// recomputes probabilities tile by tile, then applies the exact softmax
+// vector-Jacobian product).  With s = scale * q.k, P = exp(s - lse) on the
+// visible keys (0 on masked ones) and the upstream gradient dO:
+//
+//   D_i  = sum_t dO_it O_it            (= sum_j P_ij dP_ij, the row term)
+//   dP   = dO V^T,   dS = P o (dP - D)
+//   dV   = P^T dO,   dK = scale dS^T Q,   dQ = scale dS K
+//
+// Three kernels, all on the caller's stream:
+//   bwd_preprocess   D and -lse*log2(e) per row into the workspace, padded to
+//                    whole 128-row tiles (-inf / 0 on the padding, so padded
+//                    query rows carry P = 0 without a mask);
+//   bwd_dkdv         one CTA per (batch, K/V head, 128-key tile): loops over
+//                    the G query heads of the K/V head and the query tiles
+//                    that see the keys, so dK and dV of grouped heads are
+//                    summed in TMEM, not with atomics ("Grouped-Query
+//                    Attention" §5.1);
+//   bwd_dq           one CTA per (batch, head, 128-query tile): loops over
+//                    the key tiles the rows see.
+// In both tensor-core kernels warp 0 is the TMA producer, warp 1 owns TMEM
+// and issues the MMAs from one thread, warps 4-7 do the elementwise work with
+// one thread per TMEM lane (a key row in bwd_dkdv, a query row in bwd_dq).
+//
+// bwd_dkdv, TMEM columns: S^T [0,128), dP^T [128,256), dV [256,384),
+// dK [384,512).  Per query tile:
+//   S^T = K Q^T, dP^T = V dO^T        (SS MMAs, M = N = 128)
+//   P^T (16-bit) over the first 64 columns of S^T  -> dV += P^T dO  (TS MMA)
+//   dS^T (16-bit) over the first 64 columns of dP^T -> dK += dS^T Q  (TS MMA)
+// Issue order: dV(t), S^T(t+1), dK(t), dP^T(t+1): each overwrite of a TMEM
+// region follows the MMA that read it, and the next tile's exponentials
+// overlap this tile's dK and the next dP^T.
+//
+// bwd_dq, TMEM columns: S [0,128), dP [128,256), dQ [256,256+d).  Per key
+// tile: S = Q K^T, dP = dO V^T (SS), dS over the first 64 columns of dP ->
+// dQ += dS K (TS).  S(n+1) is issued as soon as the elementwise warps have
+// read S(n) into registers.
+#pragma once
+
+#include "prefill_tcgen05.cuh"
+
+namespace b200attn {
+
+struct BwdParams {
+    const void* o;
+    const void* dout;
+    const float* lse;     // [B*H, T] natural-log row statistic from the forward
+    void* dq;             // [B, H, T, d]
+    void* dk;             // [B, Hkv, T, d]
+    void* dv;             // [B, Hkv, T, d]
+    float* nl;            // workspace [B*H, Tpad]: -lse * log2(e); -inf on padding rows
+    float* dd;            // workspace [B*H, Tpad]: D = sum_t dO*O; 0 on padding rows
+    int B, H, Hkv, G, T, Tpad, d, causal;
+    int n_t;              // ceil(T / 128)
+    float scale, scale_log2;
+    uint64_t timeout_ns;
+};
+
+constexpr int kBwdThreads = 256;  // 8 warps
+
+template <int DCH> struct BwdStages {
+    static constexpr int NQ = DCH == 2 ? 2 : 4;   // bwd_dkdv: (Q, dO, nl, D) stages
+    static constexpr int NK = DCH == 2 ? 4 : 8;   // bwd_dq: K/V ring stages
+};
+
+template <int DCH>
+constexpr size_t bwd_dkdv_smem_bytes() {
+    return 1024 + size_t(2 + 2 * BwdStages<DCH>::NQ) * DCH * kChunkBytes +
+           size_t(BwdStages<DCH>::NQ) * 1024 + 256;
+}
+
+template <int DCH>
+constexpr size_t bwd_dq_smem_bytes() {
+    return 1024 + size_t(2 + BwdStages<DCH>::NK) * DCH * kChunkBytes + 256;
+}
+
+// ------------------------------------------------------------------ preprocess
+
+// D and -lse*log2(e) for every row of [B*H, Tpad]; one half-warp per row
+// (16 lanes x 8 elements cover d <= 128).
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) {
+    const int64_t rows = int64_t(p.B) * p.H * p.Tpad;
+    const int half = threadIdx.x >> 4;
+    const int hl = threadIdx.x & 15;
+    // the loop bound is uniform over the block, so every shuffle has all lanes
+    for (int64_t r0 = int64_t(blockIdx.x) * 16; r0 < rows; r0 += int64_t(gridDim.x) * 16) {
+        const int64_t r = r0 + half;
+        const bool live = r < rows;
+        const int64_t bh = live ? r / p.Tpad : 0;
+        const int i = live ? int(r - bh * p.Tpad) : p.T;
+        float acc = 0.f;
+        if (i < p.T) {
+            const size_t off = (size_t(bh) * p.T + i) * p.d;
+            const T* o = static_cast<const T*>(p.o) + off;
+            const T* g = static_cast<const T*>(p.dout) + off;
+            for (int c = hl * 8; c < p.d; c += 128) {
+                const uint4 a = *reinterpret_cast<const uint4*>(o + c);
+                const uint4 b = *reinterpret_cast<const uint4*>(g + c);
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = unpack2<T>(aw[e]), y = unpack2<T>(bw[e]);
+                    acc = fmaf(x.x, y.x, acc);
+                    acc = fmaf(x.y, y.y, acc);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 8; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+        if (live && hl == 0) {
+            p.dd[r] = i < p.T ? acc : 0.f;
+            p.nl[r] = i < p.T ? -p.lse[size_t(bh) * p.T + i] * 1.4426950408889634f : -INFINITY;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ MMA helpers
+
+// D (128 x 128, fp32 in TMEM) = A B^T with both operands K-major 128-row
+// tiles in shared memory (d/16 k-steps over the DCH 64-column chunks).
+template <int DCH>
+__device__ __forceinline__ void bwd_mma_rows(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                             int nk) {
+#pragma unroll
+    for (int kk = 0; kk < 4 * DCH; ++kk) {
+        if (kk >= nk) break;
+        const uint64_t off = uint64_t(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+        mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+// D (128 x d) (+)= A B with A (128 x 128, 16-bit) in TMEM and B a 128-row tile
+// in shared memory read MN-major (rows are the contraction index).
+__device__ __forceinline__ void bwd_mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
+                                               uint32_t idesc, bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_ts(d_tmem, a_tmem + kk * 8, b0 + uint64_t((kk * 2048) >> 4), idesc,
+               (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// 32 consecutive fp32 values of shared memory (16-byte aligned) into registers.
+__device__ __forceinline__ void lds32(const float* src, float (&r)[32]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 v = reinterpret_cast<const float4*>(src)[i];
+        r[4 * i] = v.x;
+        r[4 * i + 1] = v.y;
+        r[4 * i + 2] = v.z;
+        r[4 * i + 3] = v.w;
+    }
+}
+
+// One tile row's epilogue: 16-column pieces of a TMEM accumulator, times
+// `mul`, rounded to T and stored to `dst` (d elements) when `valid`.
+template <typename T>
+__device__ __forceinline__ void bwd_store_row(uint32_t t_acc, int d, float mul, T* dst, bool valid) {
+    for (int cc = 0; cc < d; cc += 16) {
+        uint32_t x[16];
+        tmem_ld16(t_acc + cc, x);
+        tmem_wait_ld();
+        uint4 w0, w1;
+        w0.x = pack2<T>(__uint_as_float(x[0]) * mul, __uint_as_float(x[1]) * mul);
+        w0.y = pack2<T>(__uint_as_float(x[2]) * mul, __uint_as_float(x[3]) * mul);
+        w0.z = pack2<T>(__uint_as_float(x[4]) * mul, __uint_as_float(x[5]) * mul);
+        w0.w = pack2<T>(__uint_as_float(x[6]) * mul, __uint_as_float(x[7]) * mul);
+        w1.x = pack2<T>(__uint_as_float(x[8]) * mul, __uint_as_float(x[9]) * mul);
+        w1.y = pack2<T>(__uint_as_float(x[10]) * mul, __uint_as_float(x[11]) * mul);
+        w1.z = pack2<T>(__uint_as_float(x[12]) * mul, __uint_as_float(x[13]) * mul);
+        w1.w = pack2<T>(__uint_as_float(x[14]) * mul, __uint_as_float(x[15]) * mul);
+        if (valid) {
+            reinterpret_cast<uint4*>(dst + cc)[0] = w0;
+            reinterpret_cast<uint4*>(dst + cc)[1] = w1;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ dK, dV
+
+template <typename T, int DCH>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                const BwdParams p) {
+    constexpr int NQ = BwdStages<DCH>::NQ;
+    constexpr uint32_t TB = DCH * kChunkBytes;   // one 128-row tile
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    unsigned char* base_ptr = smem_raw + (base - smem_u32(smem_raw));
+    const uint32_t sK = base, sV = base + TB;
+    const uint32_t sQ = base + 2 * TB;              // [NQ] tiles
+    const uint32_t sdO = sQ + NQ * TB;              // [NQ] tiles
+    float* rowstat = reinterpret_cast<float*>(base_ptr + (2 + 2 * NQ) * TB);  // [NQ][nl 128 | D 128]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(rowstat + NQ * 256);
+    uint64_t* kv_full = bars;            // 1
+    uint64_t* q_full = bars + 1;         // NQ
+    uint64_t* q_empty = q_full + NQ;     // NQ: the MMA commit + 4 elementwise warps
+    uint64_t* s_full = q_empty + NQ;     // 1
+    uint64_t* dp_full = s_full + 1;      // 1
+    uint64_t* p_ready = dp_full + 1;     // 1 (4 arrivals)
+    uint64_t* ds_ready = p_ready + 1;    // 1 (4 arrivals)
+    uint64_t* acc_done = ds_ready + 1;   // 1
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bk = int(blockIdx.x % unsigned(p.B * p.Hkv));
+    const int kt = int(blockIdx.x / unsigned(p.B * p.Hkv));   // heaviest (kt = 0) first
+    const int b = bk / p.Hkv, kvh = bk % p.Hkv;
+    const int q_lo = p.causal ? kt : 0;
+    const int n_q = p.n_t - q_lo;
+    const int n_it = p.G * n_q;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(kv_full), 1);
+        for (int s = 0; s < NQ; ++s) {
+            mbar_init(smem_u32(&q_full[s]), 1);
+            mbar_init(smem_u32(&q_empty[s]), 5);
+        }
+        mbar_init(smem_u32(s_full), 1);
+        mbar_init(smem_u32(dp_full), 1);
+        mbar_init(smem_u32(p_ready), 4);
+        mbar_init(smem_u32(ds_ready), 4);
+        mbar_init(smem_u32(acc_done), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmdO);
+            {
+                const uint32_t bar = smem_u32(kv_full);
+                mbar_expect_tx(bar, 2 * TB);
+                for (int c = 0; c < DCH; ++c) {
+                    tma_load_3d(sK + c * kChunkBytes, &tmK, bar, c * 64, kt * 128, bk);
+                    tma_load_3d(sV + c * kChunkBytes, &tmV, bar, c * 64, kt * 128, bk);
+                }
+            }
+            int it = 0;
+            for (; it < n_it; ++it) {
+                const int st = it % NQ;
+                if (!mbar_wait(smem_u32(&q_empty[st]), ((it / NQ) & 1) ^ 1, p.timeout_ns, abort_flag)) break;
+                const int h = kvh * p.G + it / n_q;
+                const int qt = q_lo + it % n_q;
+                const int bh = b * p.H + h;
+                const uint32_t bar = smem_u32(&q_full[st]);
+                mbar_expect_tx(bar, 2 * TB + 1024);
+                for (int c = 0; c < DCH; ++c) {
+                    tma_load_3d(sQ + st * TB + c * kChunkBytes, &tmQ, bar, c * 64, qt * 128, bh);
+                    tma_load_3d(sdO + st * TB + c * kChunkBytes, &tmdO, bar, c * 64, qt * 128, bh);
+                }
+                const size_t ro = size_t(bh) * p.Tpad + size_t(qt) * 128;
+                bulk_load(smem_u32(rowstat + st * 256), p.nl + ro, 512, bar);
+                bulk_load(smem_u32(rowstat + st * 256 + 128), p.dd + ro, 512, bar);
+            }
+            // no copy may still be landing when the CTA exits
+            mbar_wait(smem_u32(kv_full), 0, p.timeout_ns, nullptr);
+            for (int i = it - 1; i >= 0 && i >= it - NQ; --i)
+                mbar_wait(smem_u32(&q_full[i % NQ]), (i / NQ) & 1, p.timeout_ns, nullptr);
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_f16(kBF16, 128, 128, false);
+            const uint32_t idA = idesc_f16(kBF16, 128, p.d, true);
+            const int nk = p.d / 16;
+            const uint64_t aK = smem_desc_sw128(sK, 16, 1024);
+            const uint64_t aV = smem_desc_sw128(sV, 16, 1024);
+            const uint64_t bQk = smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t bdOk = smem_desc_sw128(sdO, 16, 1024);
+            const uint64_t bQm = smem_desc_sw128(sQ, kChunkBytes, 1024);
+            const uint64_t bdOm = smem_desc_sw128(sdO, kChunkBytes, 1024);
+            const auto step = [](int st) { return uint64_t(uint32_t(st) * (TB >> 4)); };
+            bool ok = mbar_wait(smem_u32(kv_full), 0, p.timeout_ns, abort_flag);
+            if (ok) ok = mbar_wait(smem_u32(&q_full[0]), 0, p.timeout_ns, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                bwd_mma_rows<DCH>(tmem, aK, bQk, idS, nk);
+                mma_commit(smem_u32(s_full));
+                bwd_mma_rows<DCH>(tmem + 128, aV, bdOk, idS, nk);
+                mma_commit(smem_u32(dp_full));
+            }
+            for (int it = 0; it < n_it && ok; ++it) {
+                const int st = it % NQ;
+                const int st1 = (it + 1) % NQ;
+                const bool more = it + 1 < n_it;
+                ok = mbar_wait(smem_u32(p_ready), it & 1, p.timeout_ns, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                bwd_mma_tmem_a(tmem + 256, tmem, bdOm + step(st), idA, it > 0);
+                if (more) {
+                    ok = mbar_wait(smem_u32(&q_full[st1]), ((it + 1) / NQ) & 1, p.timeout_ns, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    bwd_mma_rows<DCH>(tmem, aK, bQk + step(st1), idS, nk);
+                    mma_commit(smem_u32(s_full));
+                }
+                ok = mbar_wait(smem_u32(ds_ready), it & 1, p.timeout_ns, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                bwd_mma_tmem_a(tmem + 384, tmem + 128, bQm + step(st), idA, it > 0);
+                mma_commit(smem_u32(&q_empty[st]));
+                if (more) {
+                    bwd_mma_rows<DCH>(tmem + 128, aV, bdOk + step(st1), idS, nk);
+                    mma_commit(smem_u32(dp_full));
+                }
+            }
+            // every MMA issued must finish before TMEM is released
+            mma_commit(smem_u32(acc_done));
+            mbar_wait(smem_u32(acc_done), 0, p.timeout_ns, nullptr);
+        }
+    } else if (warp >= 4) {
+        // ================================================= elementwise (one key row per thread)
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t lane_base = uint32_t(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_base, tdP = tmem + lane_base + 128;
+        const float c2 = p.scale_log2;
+        bool ok = true;
+        for (int it = 0; it < n_it && ok; ++it) {
+            const int st = it % NQ;
+            const int qt = q_lo + it % n_q;
+            const float* nl = rowstat + st * 256;
+            const float* dd = nl + 128;
+            ok = mbar_wait(smem_u32(s_full), it & 1, p.timeout_ns, abort_flag);
+            if (ok) ok = mbar_wait(smem_u32(&q_full[st]), (it / NQ) & 1, p.timeout_ns, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t r[4][32];
+            tmem_ld32(tS + 0, r[0]);
+            tmem_ld32(tS + 32, r[1]);
+            tmem_ld32(tS + 64, r[2]);
+            tmem_ld32(tS + 96, r[3]);
+            tmem_wait_ld();
+            // causal diagonal tile: query column i sees key row j only when i >= j
+            const int first_vis = (p.causal && qt == kt) ? row : 0;
+            const float2 c2v = make_float2(c2, c2);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float nlv[32];
+                lds32(nl + 32 * ch, nlv);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float2 x = __ffma2_rn(make_float2(__uint_as_float(r[ch][2 * e]),
+                                                      __uint_as_float(r[ch][2 * e + 1])),
+                                          c2v, make_float2(nlv[2 * e], nlv[2 * e + 1]));
+                    if (32 * ch + 2 * e < first_vis) x.x = -INFINITY;
+                    if (32 * ch + 2 * e + 1 < first_vis) x.y = -INFINITY;
+                    const float p0 = ex2(x.x), p1 = ex2(x.y);
+                    r[ch][2 * e] = __float_as_uint(p0);
+                    r[ch][2 * e + 1] = __float_as_uint(p1);
+                    pk[e] = pack2<T>(p0, p1);
+                }
+                tmem_st16(tS + 16 * ch, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(p_ready));
+            ok = mbar_wait(smem_u32(dp_full), it & 1, p.timeout_ns, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t g[32];
+                tmem_ld32(tdP + 32 * ch, g);
+                tmem_wait_ld();
+                float ddv[32];
+                lds32(dd + 32 * ch, ddv);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float2 pp = make_float2(__uint_as_float(r[ch][2 * e]), __uint_as_float(r[ch][2 * e + 1]));
+                    const float2 t = __fadd2_rn(make_float2(__uint_as_float(g[2 * e]), __uint_as_float(g[2 * e + 1])),
+                                                make_float2(-ddv[2 * e], -ddv[2 * e + 1]));
+                    const float2 ds = __fmul2_rn(pp, t);
+                    pk[e] = pack2<T>(ds.x, ds.y);
+                }
+                // columns [16ch, 16ch+16) of the dP^T region were read with chunks <= ch
+                tmem_st16(tdP + 16 * ch, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(smem_u32(ds_ready));
+                mbar_arrive(smem_u32(&q_empty[st]));
+            }
+        }
+        // ---- epilogue: dV and scale * dK rows of this key tile
+        if (ok) ok = mbar_wait(smem_u32(acc_done), 0, p.timeout_ns, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc_fence_after();
+            const int j = kt * 128 + row;
+            const bool valid = j < p.T;
+            const size_t orow = (size_t(bk) * p.T + (valid ? j : 0)) * p.d;
+            bwd_store_row<T>(tmem + lane_base + 256, p.d, 1.f, static_cast<T*>(p.dv) + orow, valid);
+            bwd_store_row<T>(tmem + lane_base + 384, p.d, p.scale, static_cast<T*>(p.dk) + orow, valid);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ dQ
+
+template <typename T, int DCH>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+              const BwdParams p) {
+    constexpr int NK = BwdStages<DCH>::NK;
+    constexpr uint32_t TB = DCH * kChunkBytes;
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    unsigned char* base_ptr = smem_raw + (base - smem_u32(smem_raw));
+    const uint32_t sQ = base, sdO = base + TB;
+    const uint32_t sRing = base + 2 * TB;           // [NK] tiles: K_0, V_0, K_1, V_1, ...
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + (2 + NK) * TB);
+    uint64_t* q_full = bars;             // 1
+    uint64_t* kv_full = bars + 1;        // NK
+    uint64_t* kv_empty = kv_full + NK;   // NK
+    uint64_t* s_full = kv_empty + NK;    // 1
+    uint64_t* dp_full = s_full + 1;      // 1
+    uint64_t* s_read = dp_full + 1;      // 1 (4 arrivals)
+    uint64_t* ds_ready = s_read + 1;     // 1 (4 arrivals)
+    uint64_t* acc_done = ds_ready + 1;   // 1
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = int(blockIdx.x % unsigned(p.B * p.H));
+    const int qt = p.n_t - 1 - int(blockIdx.x / unsigned(p.B * p.H));   // heaviest first
+    const int b = bh / p.H, h = bh % p.H;
+    const int bk = b * p.Hkv + h / p.G;
+    const int n_kv = p.causal ? qt + 1 : p.n_t;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(q_full), 1);
+        for (int s = 0; s < NK; ++s) {
+            mbar_init(smem_u32(&kv_full[s]), 1);
+            mbar_init(smem_u32(&kv_empty[s]), 1);
+        }
+        mbar_init(smem_u32(s_full), 1);
+        mbar_init(smem_u32(dp_full), 1);
+        mbar_init(smem_u32(s_read), 4);
+        mbar_init(smem_u32(ds_ready), 4);
+        mbar_init(smem_u32(acc_done), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            {
+                const uint32_t bar = smem_u32(q_full);
+                mbar_expect_tx(bar, 2 * TB);
+                for (int c = 0; c < DCH; ++c) {
+                    tma_load_3d(sQ + c * kChunkBytes, &tmQ, bar, c * 64, qt * 128, bh);
+                    tma_load_3d(sdO + c * kChunkBytes, &tmdO, bar, c * 64, qt * 128, bh);
+                }
+            }
+            const int n_loads = 2 * n_kv;
+            int li = 0;
+            for (; li < n_loads; ++li) {
+                const int st = li % NK;
+                if (!mbar_wait(smem_u32(&kv_empty[st]), ((li / NK) & 1) ^ 1, p.timeout_ns, abort_flag)) break;
+                const uint32_t bar = smem_u32(&kv_full[st]);
+                mbar_expect_tx(bar, TB);
+                const CUtensorMap* map = (li & 1) ? &tmV : &tmK;
+                for (int c = 0; c < DCH; ++c)
+                    tma_load_3d(sRing + st * TB + c * kChunkBytes, map, bar, c * 64, (li >> 1) * 128, bk);
+            }
+            mbar_wait(smem_u32(q_full), 0, p.timeout_ns, nullptr);
+            for (int i = li - 1; i >= 0 && i >= li - NK; --i)
+                mbar_wait(smem_u32(&kv_full[i % NK]), (i / NK) & 1, p.timeout_ns, nullptr);
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_f16(kBF16, 128, 128, false);
+            const uint32_t idA = idesc_f16(kBF16, 128, p.d, true);
+            const int nk = p.d / 16;
+            const uint64_t aQ = smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t adO = smem_desc_sw128(sdO, 16, 1024);
+            const uint64_t bRk = smem_desc_sw128(sRing, 16, 1024);
+            const uint64_t bRm = smem_desc_sw128(sRing, kChunkBytes, 1024);
+            const auto step = [](int st) { return uint64_t(uint32_t(st) * (TB >> 4)); };
+            const auto full = [&](int li) {
+                return mbar_wait(smem_u32(&kv_full[li % NK]), (li / NK) & 1, p.timeout_ns, abort_flag);
+            };
+            bool ok = mbar_wait(smem_u32(q_full), 0, p.timeout_ns, abort_flag);
+            if (ok) ok = full(0);
+            if (ok) {
+                tc_fence_after();
+                bwd_mma_rows<DCH>(tmem, aQ, bRk + step(0), idS, nk);
+                mma_commit(smem_u32(s_full));
+                ok = full(1);
+            }
+            if (ok) {
+                tc_fence_after();
+                bwd_mma_rows<DCH>(tmem + 128, adO, bRk + step(1 % NK), idS, nk);
+                mma_commit(smem_u32(dp_full));
+                mma_commit(smem_u32(&kv_empty[1 % NK]));
+            }
+            for (int n = 0; n < n_kv && ok; ++n) {
+                const bool more = n + 1 < n_kv;
+                const int liK = 2 * n;
+                ok = mbar_wait(smem_u32(s_read), n & 1, p.timeout_ns, abort_flag);
+                if (!ok) break;
+                if (more) {
+                    ok = full(liK + 2);
+                    if (!ok) break;
+                    tc_fence_after();
+                    bwd_mma_rows<DCH>(tmem, aQ, bRk + step((liK + 2) % NK), idS, nk);
+                    mma_commit(smem_u32(s_full));
+                }
+                ok = mbar_wait(smem_u32(ds_ready), n & 1, p.timeout_ns, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                bwd_mma_tmem_a(tmem + 256, tmem + 128, bRm + step(liK % NK), idA, n > 0);
+                mma_commit(smem_u32(&kv_empty[liK % NK]));
+                if (more) {
+                    ok = full(liK + 3);
+                    if (!ok) break;
+                    tc_fence_after();
+                    bwd_mma_rows<DCH>(tmem + 128, adO, bRk + step((liK + 3) % NK), idS, nk);
+                    mma_commit(smem_u32(dp_full));
+                    mma_commit(smem_u32(&kv_empty[(liK + 3) % NK]));
+                }
+            }
+            mma_commit(smem_u32(acc_done));
+            mbar_wait(smem_u32(acc_done), 0, p.timeout_ns, nullptr);
+        }
+    } else if (warp >= 4) {
+        // ================================================= elementwise (one query row per thread)
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t lane_base = uint32_t(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_base, tdP = tmem + lane_base + 128;
+        const int i = qt * 128 + row;
+        const size_t ro = size_t(bh) * p.Tpad + size_t(i);
+        const float nl = p.nl[ro];
+        const float dd = p.dd[ro];
+        const float c2 = p.scale_log2;
+        bool ok = true;
+        for (int n = 0; n < n_kv && ok; ++n) {
+            ok = mbar_wait(smem_u32(s_full), n & 1, p.timeout_ns, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t r[4][32];
+            tmem_ld32(tS + 0, r[0]);
+            tmem_ld32(tS + 32, r[1]);
+            tmem_ld32(tS + 64, r[2]);
+            tmem_ld32(tS + 96, r[3]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(s_read));
+            // key j = 128 n + c is visible when j < T and (not causal or j <= i)
+            int last = 127;
+            if (n * 128 + 127 >= p.T) last = p.T - 1 - n * 128;
+            if (p.causal && n == qt) last = min(last, row);
+            const float2 c2v = make_float2(c2, c2);
+            const float2 nlv = make_float2(nl, nl);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float2 x = __ffma2_rn(make_float2(__uint_as_float(r[ch][2 * e]),
+                                                      __uint_as_float(r[ch][2 * e + 1])),
+                                          c2v, nlv);
+                    if (32 * ch + 2 * e > last) x.x = -INFINITY;
+                    if (32 * ch + 2 * e + 1 > last) x.y = -INFINITY;
+                    r[ch][2 * e] = __float_as_uint(ex2(x.x));
+                    r[ch][2 * e + 1] = __float_as_uint(ex2(x.y));
+                }
+            ok = mbar_wait(smem_u32(dp_full), n & 1, p.timeout_ns, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const float2 ndd = make_float2(-dd, -dd);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t g[32];
+                tmem_ld32(tdP + 32 * ch, g);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float2 pp = make_float2(__uint_as_float(r[ch][2 * e]), __uint_as_float(r[ch][2 * e + 1]));
+                    const float2 t = __fadd2_rn(make_float2(__uint_as_float(g[2 * e]), __uint_as_float(g[2 * e + 1])), ndd);
+                    const float2 ds = __fmul2_rn(pp, t);
+                    pk[e] = pack2<T>(ds.x, ds.y);
+                }
+                tmem_st16(tdP + 16 * ch, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(ds_ready));
+        }
+        if (ok) ok = mbar_wait(smem_u32(acc_done), 0, p.timeout_ns, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc_fence_after();
+            const bool valid = i < p.T;
+            const size_t orow = (size_t(bh) * p.T + (valid ? i : 0)) * p.d;
+            bwd_store_row<T>(tmem + lane_base + 256, p.d, p.scale, static_cast<T*>(p.dq) + orow, valid);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace b200attn

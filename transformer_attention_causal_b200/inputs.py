@@ -4,7 +4,8 @@ This module holds no attention arithmetic: it only draws i.i.d. N(0, 1)
 numbers and rounds them to the requested dtype.
 
 Recipe.  A tensor of shape [B, Hx, L, d] is filled one (b, hx) slice at a time.
-Slice (b, hx) of stream ``stream`` (0 = Q, 1 = K, 2 = V, others free) is
+Slice (b, hx) of stream ``stream`` (0 = Q, 1 = K, 2 = V, 3 = the upstream
+gradient dO of the backward pass, others free) is
 ``torch.randn((L, d), generator=torch.Generator().manual_seed(slice_seed))`` in
 float32, then cast to the dtype with round-to-nearest-even, where
 ``slice_seed = splitmix64(seed, stream, b, hx) >> 1``.  Because every slice
@@ -22,7 +23,7 @@ from concurrent.futures import ThreadPoolExecutor
 import torch
 
 _MASK = (1 << 64) - 1
-Q_STREAM, K_STREAM, V_STREAM = 0, 1, 2
+Q_STREAM, K_STREAM, V_STREAM, DO_STREAM = 0, 1, 2, 3
 
 
 def _splitmix64(x: int) -> int:
@@ -77,3 +78,8 @@ def qkv(B: int, H: int, Hkv: int, Tq: int, S: int, d: int, dtype: torch.dtype,
         k = torch.cat([k, pad], dim=2)
         v = torch.cat([v, pad], dim=2)
     return q, k, v
+
+
+def upstream(B: int, H: int, T: int, d: int, dtype: torch.dtype, seed: int = 0) -> torch.Tensor:
+    """dO [B, H, T, d] on the CPU: the gradient fed into the backward pass."""
+    return normal((B, H, T, d), seed, DO_STREAM, dtype)
