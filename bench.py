@@ -7,10 +7,11 @@ One step = one call of the library on one batch of the workload (default: the
 BitNet-3B-shaped causal MHA prefill, B=1, H=32, T=2048, d=80, bf16).  The
 line also carries the cached-decode half of the metric (GQA decode, B=64,
 H=32/8, S=8192, d=128, bf16), the same decode over a paged cache (64-token
-pages), the GQA prefill with a 2048-key local window (B=2, T=8192), and the
+pages), the GQA prefill with a 2048-key local window (B=2, T=8192), the
 KV-cache append with RoPE on K of the GQA prefill's keys and values (B=8,
-Hkv=8, 4096 tokens, d=128, bf16), each measured the same way with its own
-roofline.
+Hkv=8, 4096 tokens, d=128, bf16), and the backward pass of the GQA prefill
+(dQ, dK, dV from the forward's O and row statistic), each measured the same
+way with its own roofline.
 
 Timing: W untimed steps, then exactly K timed steps bracketed by a barrier and
 torch.cuda.synchronize() on both sides.  Before every timed call L2 is flushed
@@ -60,6 +61,9 @@ WORKLOADS = {
     # the GQA decode over a paged cache: 64-token pages in a seeded physical order
     "gqa_decode_paged_bf16": dict(kind="paged", dtype="bf16", B=64, H=32, Hkv=8, Tnew=1,
                                   start=8191, S=8192, d=128, page=64),
+    # the backward pass of the GQA prefill (its forward runs untimed during setup)
+    "gqa16x8_backward_bf16": dict(kind="backward", dtype="bf16", B=8, H=16, Hkv=8, T=4096,
+                                  d=128),
     # the step before attention: the GQA prefill's 4096 new keys (RoPE) and values
     # written into an empty cache
     "kv_append_rope_gqa16x8_bf16": dict(kind="append", dtype="bf16", B=8, H=16, Hkv=8,
@@ -70,24 +74,30 @@ DECODE_WORKLOAD = "gqa_decode_bf16"
 APPEND_WORKLOAD = "kv_append_rope_gqa16x8_bf16"
 WINDOW_WORKLOAD = "gqa_prefill_swa_bf16"
 PAGED_WORKLOAD = "gqa_decode_paged_bf16"
+BACKWARD_WORKLOAD = "gqa16x8_backward_bf16"
 TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
 KERNEL_SOURCES = {"tcgen05": "prefill_tcgen05.cuh", "splitkv": "decode_splitkv.cuh",
                   "paged": "decode_splitkv.cuh",
-                  "simt": "simt_attn.cuh", "append": "kv_append.cuh"}
+                  "simt": "simt_attn.cuh", "append": "kv_append.cuh",
+                  "backward": "prefill_backward.cuh"}
 
 
 # ------------------------------------------------------------------ workload algebra
 
+def full_sequence(w):
+    return w["kind"] in ("prefill", "backward")
+
+
 def q_len(w):
-    return w["T"] if w["kind"] == "prefill" else w["Tnew"]
+    return w["T"] if full_sequence(w) else w["Tnew"]
 
 
 def kv_len(w):
-    return w["T"] if w["kind"] == "prefill" else w["S"]
+    return w["T"] if full_sequence(w) else w["S"]
 
 
 def start_pos(w):
-    return 0 if w["kind"] == "prefill" else w["start"]
+    return 0 if full_sequence(w) else w["start"]
 
 
 def visible_pairs(w):
@@ -100,10 +110,17 @@ def visible_pairs(w):
     return Tq * s0 + Tq * (Tq + 1) // 2
 
 
+def flops_per_pair(w):
+    """Forward: 4*d per visible (query, key) pair per query head (2*d for Q.K,
+    2*d for P.V).  Backward: 10*d (the five products S, dP, dV, dK, dQ); the
+    second recomputation of S and dP in the dQ kernel is not credited."""
+    return (10 if w["kind"] == "backward" else 4) * w["d"]
+
+
 def algorithmic_flops(w):
-    """4*d FLOPs per visible (query, key) pair per query head (2*d for Q.K, 2*d
-    for P.V); masked pairs, exponentials and maxima are not counted."""
-    return 4 * w["d"] * w["B"] * w["H"] * visible_pairs(w)
+    """FLOPs of the visible pairs; masked pairs, exponentials and maxima are
+    not counted."""
+    return flops_per_pair(w) * w["B"] * w["H"] * visible_pairs(w)
 
 
 def esize(w):
@@ -130,8 +147,10 @@ def bound(w):
 def config_of(name, w, world):
     cfg = {"workload": name, "B": w["B"], "H": w["H"], "Hkv": w["Hkv"], "d": w["d"],
            "dtype": w["dtype"], "causal": True, "scale": f"1/sqrt({w['d']})"}
-    if w["kind"] == "prefill":
+    if full_sequence(w):
         cfg["T"] = w["T"]
+        if w["kind"] == "backward":
+            cfg["pass"] = "backward: dq, dk, dv from q, k, v, o, lse, dout"
         if w.get("window"):
             cfg["window"] = w["window"]
     elif w["kind"] == "paged":
@@ -282,6 +301,20 @@ class Case:
             self.kernel, self.launches, self.device = "append", 1, device
             return
         q, k, v = inputs.qkv(w["B"], w["H"], w["Hkv"], Tq, S, w["d"], dt, seed=seed)
+        if w["kind"] == "backward":
+            self.scale = 1.0 / math.sqrt(w["d"])
+            dout = inputs.upstream(w["B"], w["H"], Tq, w["d"], dt, seed=seed)
+            qd, kd, vd = (t.to(device) for t in (q, k, v))
+            lse = torch.empty((w["B"], w["H"], Tq), dtype=torch.float32, device=device)
+            o = attn.prefill(qd, kd, vd, scale=self.scale, causal=True, lse=lse)
+            self.host = [t.pin_memory() for t in (q, k, v, o.cpu(), lse.cpu(), dout)]
+            self.dev_in = [qd, kd, vd, o, lse, dout.to(device)]
+            self.dev_out = [torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)]
+            self.host_out = [torch.empty(t.shape, dtype=dt).pin_memory() for t in self.dev_out]
+            need = attn.prefill_backward_workspace_size(dt, w["B"], w["H"], w["Hkv"], Tq, w["d"])
+            self.ws = torch.empty(need, dtype=torch.uint8, device=device)
+            self.kernel, self.launches, self.device = "backward", 3, device
+            return
         if w["kind"] == "paged":
             # pages [B * S / P, Hkv, P, d] in a seeded physical order, and the table
             P, n = w["page"], S // w["page"]
@@ -324,6 +357,10 @@ class Case:
         if w["kind"] == "append":
             self.attn.kv_append_rope(*self.dev_in, *self.dev_out, start_pos=w["start"],
                                      rope_base=w["base"])
+        elif w["kind"] == "backward":
+            dq, dk, dv = self.dev_out
+            self.attn.prefill_backward(*self.dev_in, scale=self.scale, causal=True, dq=dq, dk=dk,
+                                       dv=dv, workspace=self.ws)
         elif w["kind"] == "prefill":
             self.attn.prefill(self.q, self.k, self.v, scale=self.scale, causal=True, out=self.out,
                               window=w.get("window", 0))
@@ -467,6 +504,12 @@ class OracleSample:
                                                 w["d"], dt, seed=seed)
             self.total = w["B"]
             self.what = "sequences (paged, all heads) of"
+        elif w["kind"] == "backward":
+            self.q, self.k, self.v = inputs.qkv(w["B"], w["H"], w["Hkv"], q_len(w), kv_len(w),
+                                                w["d"], dt, seed=seed)
+            self.dout = inputs.upstream(w["B"], w["H"], q_len(w), w["d"], dt, seed=seed)
+            self.total = w["B"] * w["H"]
+            self.what = "(batch, head) slices (full backward of one head) of"
         else:
             self.q, self.k, self.v = inputs.qkv(w["B"], w["H"], w["Hkv"], q_len(w), kv_len(w),
                                                 w["d"], dt, seed=seed)
@@ -497,6 +540,20 @@ class OracleSample:
             for kn, vn, pos in jobs:
                 rope_append(kn, vn, start_pos=pos, base=w["base"])
             return time.perf_counter() - t0, n * self.per_unit, n
+        if w["kind"] == "backward":
+            from oracle import attention_backward
+
+            G = w["H"] // w["Hkv"]
+            secs = 0.0
+            for idx in rng.choice(self.total, size=n, replace=False):
+                b, h = divmod(int(idx), w["H"])
+                kvh = h // G
+                t0 = time.perf_counter()
+                attention_backward(self.q[b:b + 1, h:h + 1], self.k[b:b + 1, kvh:kvh + 1],
+                                   self.v[b:b + 1, kvh:kvh + 1], self.dout[b:b + 1, h:h + 1],
+                                   scale=1 / math.sqrt(w["d"]))
+                secs += time.perf_counter() - t0
+            return secs, n * self.per_unit, n
         if w["kind"] == "paged":
             from oracle import paged_attention
 
@@ -531,7 +588,7 @@ class OracleSample:
         """Rows that take the oracle about target_s seconds, from a pilot run."""
         from oracle import num_cores
 
-        secs, work, _ = self.run(4 * num_cores(), rng)
+        secs, work, _ = self.run(1 if self.w["kind"] == "backward" else 4 * num_cores(), rng)
         return int(min(self.total, max(16, target_s * (work / max(secs, 1e-6)) / self.per_unit)))
 
 
@@ -616,7 +673,8 @@ def run_ours(args, dist_ctx):
         "device_status": status,
     }
     legs = [] if args.no_decode else [("decode", DECODE_WORKLOAD), ("paged", PAGED_WORKLOAD),
-                                      ("window", WINDOW_WORKLOAD), ("append", APPEND_WORKLOAD)]
+                                      ("window", WINDOW_WORKLOAD), ("append", APPEND_WORKLOAD),
+                                      ("backward", BACKWARD_WORKLOAD)]
     del case
     for key, leg in legs:
         if leg == name:
