@@ -25,8 +25,14 @@
 //   bwd_dq           one CTA per (batch, head, 128-query tile): loops over
 //                    the key tiles the rows see.
 // In both tensor-core kernels warp 0 is the TMA producer, warp 1 owns TMEM
-// and issues the MMAs from one thread, warps 4-7 do the elementwise work with
-// one thread per TMEM lane (a key row in bwd_dkdv, a query row in bwd_dq).
+// and issues the MMAs from one thread, warps 4-11 do the elementwise work:
+// one TMEM lane (a key row in bwd_dkdv, a query row in bwd_dq) per thread,
+// warps 4-7 on the tile's columns 0-63 and warps 8-11 on columns 64-127 (no
+// step of the backward reduces along a row, so the halves never meet).
+// 16-bit P / dS values of columns 64h..64h+63 are packed into TMEM columns
+// 64h..64h+31 of the region they were read from, so a half never overwrites
+// scores the other half has yet to read; the TS MMAs' A operand follows that
+// map (k-steps 4-7 start 32 columns further on).
 //
 // bwd_dkdv, TMEM columns: S^T [0,128), dP^T [128,256), dV [256,384),
 // dK [384,512).  Per query tile:
@@ -37,10 +43,13 @@
 // region follows the MMA that read it, and the next tile's exponentials
 // overlap this tile's dK and the next dP^T.
 //
-// bwd_dq, TMEM columns: S [0,128), dP [128,256), dQ [256,256+d).  Per key
-// tile: S = Q K^T, dP = dO V^T (SS), dS over the first 64 columns of dP ->
-// dQ += dS K (TS).  S(n+1) is issued as soon as the elementwise warps have
-// read S(n) into registers.
+// bwd_dq, TMEM columns: S [0,128), dP [128,256), dQ [256,256+d), dS (16-bit
+// pairs) [384,448), Q (16-bit pairs, copied in once by the elementwise warps)
+// [448,512).  Per key tile: S = Q K^T (TS: Q from TMEM), dP = dO V^T (SS),
+// dQ += dS K (TS).  Every shared-memory operand read competes with the TMA
+// copies for the SM's 128 B/clk, so Q comes from TMEM; and because dS has
+// its own columns, S(n+1) and dP(n+1) are issued as soon as the elementwise
+// warps have read S(n) and dP(n) into registers.
 #pragma once
 
 #include "prefill_tcgen05.cuh"
@@ -62,11 +71,15 @@ struct BwdParams {
     uint64_t timeout_ns;
 };
 
-constexpr int kBwdThreads = 256;  // 8 warps
+constexpr int kBwdThreads = 384;  // 12 warps: producer, MMA, 2 idle, 8 elementwise
 
+// Ring depths, as deep as shared memory allows.  In bwd_dq a K tile is read
+// from S(n) until dQ(n), a V tile only by dP(n): separate rings, the K ring
+// the deeper.
 template <int DCH> struct BwdStages {
-    static constexpr int NQ = DCH == 2 ? 2 : 4;   // bwd_dkdv: (Q, dO, nl, D) stages
-    static constexpr int NK = DCH == 2 ? 4 : 8;   // bwd_dq: K/V ring stages
+    static constexpr int NQ = DCH == 2 ? 2 : 5;    // bwd_dkdv: (Q, dO, nl, D) stages
+    static constexpr int NKR = DCH == 2 ? 3 : 6;   // bwd_dq: K stages (read by S(n) and dQ(n))
+    static constexpr int NVR = DCH == 2 ? 2 : 4;   // bwd_dq: V stages (read by dP(n) only)
 };
 
 template <int DCH>
@@ -77,7 +90,7 @@ constexpr size_t bwd_dkdv_smem_bytes() {
 
 template <int DCH>
 constexpr size_t bwd_dq_smem_bytes() {
-    return 1024 + size_t(2 + BwdStages<DCH>::NK) * DCH * kChunkBytes + 256;
+    return 1024 + size_t(2 + BwdStages<DCH>::NKR + BwdStages<DCH>::NVR) * DCH * kChunkBytes + 256;
 }
 
 // ------------------------------------------------------------------ preprocess
@@ -137,32 +150,35 @@ __device__ __forceinline__ void bwd_mma_rows(uint32_t d_tmem, uint64_t a0, uint6
 }
 
 // D (128 x d) (+)= A B with A (128 x 128, 16-bit) in TMEM and B a 128-row tile
-// in shared memory read MN-major (rows are the contraction index).
+// in shared memory read MN-major (rows are the contraction index).  A's
+// contraction columns 0-63 sit in TMEM columns 0-31, columns 64-127 in TMEM
+// columns 64-95 (each elementwise half packs into its own range).
 __device__ __forceinline__ void bwd_mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
                                                uint32_t idesc, bool accumulate) {
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-        mma_ts(d_tmem, a_tmem + kk * 8, b0 + uint64_t((kk * 2048) >> 4), idesc,
+        mma_ts(d_tmem, a_tmem + kk * 8 + (kk >= 4 ? 32 : 0), b0 + uint64_t((kk * 2048) >> 4), idesc,
                (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// 32 consecutive fp32 values of shared memory (16-byte aligned) into registers.
-__device__ __forceinline__ void lds32(const float* src, float (&r)[32]) {
+// 32 consecutive fp32 values of shared memory (16-byte aligned shared
+// address) into registers, 16 bytes per load (every lane reads the same
+// address: one broadcast per load).
+__device__ __forceinline__ void lds32(uint32_t saddr, float (&r)[32]) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float4 v = reinterpret_cast<const float4*>(src)[i];
-        r[4 * i] = v.x;
-        r[4 * i + 1] = v.y;
-        r[4 * i + 2] = v.z;
-        r[4 * i + 3] = v.w;
-    }
+    for (int i = 0; i < 8; ++i)
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(r[4 * i]), "=f"(r[4 * i + 1]), "=f"(r[4 * i + 2]), "=f"(r[4 * i + 3])
+                     : "r"(saddr + 16 * i));
 }
 
-// One tile row's epilogue: 16-column pieces of a TMEM accumulator, times
-// `mul`, rounded to T and stored to `dst` (d elements) when `valid`.
+// One tile row's epilogue: 16-column pieces first, first + step, ... of a
+// TMEM accumulator, times `mul`, rounded to T and stored to `dst` (d
+// elements) when `valid`.
 template <typename T>
-__device__ __forceinline__ void bwd_store_row(uint32_t t_acc, int d, float mul, T* dst, bool valid) {
-    for (int cc = 0; cc < d; cc += 16) {
+__device__ __forceinline__ void bwd_store_row(uint32_t t_acc, int d, float mul, T* dst, bool valid,
+                                              int first = 0, int step = 16) {
+    for (int cc = first; cc < d; cc += step) {
         uint32_t x[16];
         tmem_ld16(t_acc + cc, x);
         tmem_wait_ld();
@@ -202,11 +218,11 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     uint64_t* bars = reinterpret_cast<uint64_t*>(rowstat + NQ * 256);
     uint64_t* kv_full = bars;            // 1
     uint64_t* q_full = bars + 1;         // NQ
-    uint64_t* q_empty = q_full + NQ;     // NQ: the MMA commit + 4 elementwise warps
+    uint64_t* q_empty = q_full + NQ;     // NQ: the MMA commit + 8 elementwise warps
     uint64_t* s_full = q_empty + NQ;     // 1
     uint64_t* dp_full = s_full + 1;      // 1
-    uint64_t* p_ready = dp_full + 1;     // 1 (4 arrivals)
-    uint64_t* ds_ready = p_ready + 1;    // 1 (4 arrivals)
+    uint64_t* p_ready = dp_full + 1;     // 1 (8 arrivals)
+    uint64_t* ds_ready = p_ready + 1;    // 1 (8 arrivals)
     uint64_t* acc_done = ds_ready + 1;   // 1
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -224,12 +240,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(smem_u32(kv_full), 1);
         for (int s = 0; s < NQ; ++s) {
             mbar_init(smem_u32(&q_full[s]), 1);
-            mbar_init(smem_u32(&q_empty[s]), 5);
+            mbar_init(smem_u32(&q_empty[s]), 9);
         }
         mbar_init(smem_u32(s_full), 1);
         mbar_init(smem_u32(dp_full), 1);
-        mbar_init(smem_u32(p_ready), 4);
-        mbar_init(smem_u32(ds_ready), 4);
+        mbar_init(smem_u32(p_ready), 8);
+        mbar_init(smem_u32(ds_ready), 8);
         mbar_init(smem_u32(acc_done), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -332,34 +348,33 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     } else if (warp >= 4) {
         // ================================================= elementwise (one key row per thread)
         const int wq = warp & 3;
+        const int half = (warp - 4) >> 2;         // query columns 64*half .. 64*half + 63
         const int row = wq * 32 + lane;
         const uint32_t lane_base = uint32_t(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_base, tdP = tmem + lane_base + 128;
+        const uint32_t tS = tmem + lane_base + 64 * half, tdP = tmem + lane_base + 128 + 64 * half;
         const float c2 = p.scale_log2;
         bool ok = true;
         for (int it = 0; it < n_it && ok; ++it) {
             const int st = it % NQ;
             const int qt = q_lo + it % n_q;
-            const float* nl = rowstat + st * 256;
-            const float* dd = nl + 128;
+            const uint32_t nl = smem_u32(rowstat + st * 256 + 64 * half);
+            const uint32_t dd = nl + 128 * 4;
             ok = mbar_wait(smem_u32(s_full), it & 1, p.timeout_ns, abort_flag);
             if (ok) ok = mbar_wait(smem_u32(&q_full[st]), (it / NQ) & 1, p.timeout_ns, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            uint32_t r[4][32];
+            uint32_t r[2][32];
             tmem_ld32(tS + 0, r[0]);
             tmem_ld32(tS + 32, r[1]);
-            tmem_ld32(tS + 64, r[2]);
-            tmem_ld32(tS + 96, r[3]);
             tmem_wait_ld();
             // causal diagonal tile: query column i sees key row j only when i >= j
-            const int first_vis = (p.causal && qt == kt) ? row : 0;
+            const int first_vis = ((p.causal && qt == kt) ? row : 0) - 64 * half;
             const float2 c2v = make_float2(c2, c2);
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 float nlv[32];
-                lds32(nl + 32 * ch, nlv);
+                lds32(nl + 128 * ch, nlv);
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -373,6 +388,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     r[ch][2 * e + 1] = __float_as_uint(p1);
                     pk[e] = pack2<T>(p0, p1);
                 }
+                // columns [16ch, 16ch+16) of this half were read with chunk 0
                 tmem_st16(tS + 16 * ch, pk);
             }
             tmem_wait_st();
@@ -384,12 +400,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 uint32_t g[32];
                 tmem_ld32(tdP + 32 * ch, g);
                 tmem_wait_ld();
                 float ddv[32];
-                lds32(dd + 32 * ch, ddv);
+                lds32(dd + 128 * ch, ddv);
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -399,7 +415,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     const float2 ds = __fmul2_rn(pp, t);
                     pk[e] = pack2<T>(ds.x, ds.y);
                 }
-                // columns [16ch, 16ch+16) of the dP^T region were read with chunks <= ch
+                // columns [16ch, 16ch+16) of this half were read with chunks <= ch
                 tmem_st16(tdP + 16 * ch, pk);
             }
             tmem_wait_st();
@@ -418,8 +434,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int j = kt * 128 + row;
             const bool valid = j < p.T;
             const size_t orow = (size_t(bk) * p.T + (valid ? j : 0)) * p.d;
-            bwd_store_row<T>(tmem + lane_base + 256, p.d, 1.f, static_cast<T*>(p.dv) + orow, valid);
-            bwd_store_row<T>(tmem + lane_base + 384, p.d, p.scale, static_cast<T*>(p.dk) + orow, valid);
+            if (half == 0)
+                bwd_store_row<T>(tmem + lane_base + 256, p.d, 1.f, static_cast<T*>(p.dv) + orow, valid);
+            else
+                bwd_store_row<T>(tmem + lane_base + 384, p.d, p.scale, static_cast<T*>(p.dk) + orow, valid);
         }
     }
 
@@ -438,23 +456,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
               const BwdParams p) {
-    constexpr int NK = BwdStages<DCH>::NK;
+    constexpr int NKR = BwdStages<DCH>::NKR;
+    constexpr int NVR = BwdStages<DCH>::NVR;
     constexpr uint32_t TB = DCH * kChunkBytes;
     constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char* base_ptr = smem_raw + (base - smem_u32(smem_raw));
     const uint32_t sQ = base, sdO = base + TB;
-    const uint32_t sRing = base + 2 * TB;           // [NK] tiles: K_0, V_0, K_1, V_1, ...
-    uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + (2 + NK) * TB);
+    const uint32_t sK = base + 2 * TB;              // [NKR] K tiles
+    const uint32_t sV = sK + NKR * TB;              // [NVR] V tiles
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + (2 + NKR + NVR) * TB);
     uint64_t* q_full = bars;             // 1
-    uint64_t* kv_full = bars + 1;        // NK
-    uint64_t* kv_empty = kv_full + NK;   // NK
-    uint64_t* s_full = kv_empty + NK;    // 1
+    uint64_t* k_full = bars + 1;         // NKR
+    uint64_t* k_empty = k_full + NKR;    // NKR
+    uint64_t* v_full = k_empty + NKR;    // NVR
+    uint64_t* v_empty = v_full + NVR;    // NVR
+    uint64_t* s_full = v_empty + NVR;    // 1
     uint64_t* dp_full = s_full + 1;      // 1
-    uint64_t* s_read = dp_full + 1;      // 1 (4 arrivals)
-    uint64_t* ds_ready = s_read + 1;     // 1 (4 arrivals)
-    uint64_t* acc_done = ds_ready + 1;   // 1
+    uint64_t* s_read = dp_full + 1;      // 1 (8 arrivals): S(n) in registers
+    uint64_t* dp_read = s_read + 1;      // 1 (8 arrivals): dP(n) in registers
+    uint64_t* ds_ready = dp_read + 1;    // 1 (8 arrivals): dS(n) in TMEM
+    uint64_t* ds_free = ds_ready + 1;    // 1: dQ(n) has read dS(n)
+    uint64_t* q_tmem = ds_free + 1;      // 1 (8 arrivals): Q copied into TMEM
+    uint64_t* acc_done = q_tmem + 1;     // 1
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -468,14 +493,21 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(q_full), 1);
-        for (int s = 0; s < NK; ++s) {
-            mbar_init(smem_u32(&kv_full[s]), 1);
-            mbar_init(smem_u32(&kv_empty[s]), 1);
+        for (int s = 0; s < NKR; ++s) {
+            mbar_init(smem_u32(&k_full[s]), 1);
+            mbar_init(smem_u32(&k_empty[s]), 1);
+        }
+        for (int s = 0; s < NVR; ++s) {
+            mbar_init(smem_u32(&v_full[s]), 1);
+            mbar_init(smem_u32(&v_empty[s]), 1);
         }
         mbar_init(smem_u32(s_full), 1);
         mbar_init(smem_u32(dp_full), 1);
-        mbar_init(smem_u32(s_read), 4);
-        mbar_init(smem_u32(ds_ready), 4);
+        mbar_init(smem_u32(s_read), 8);
+        mbar_init(smem_u32(dp_read), 8);
+        mbar_init(smem_u32(ds_ready), 8);
+        mbar_init(smem_u32(ds_free), 1);
+        mbar_init(smem_u32(q_tmem), 8);
         mbar_init(smem_u32(acc_done), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -502,20 +534,33 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tma_load_3d(sdO + c * kChunkBytes, &tmdO, bar, c * 64, qt * 128, bh);
                 }
             }
-            const int n_loads = 2 * n_kv;
-            int li = 0;
-            for (; li < n_loads; ++li) {
-                const int st = li % NK;
-                if (!mbar_wait(smem_u32(&kv_empty[st]), ((li / NK) & 1) ^ 1, p.timeout_ns, abort_flag)) break;
-                const uint32_t bar = smem_u32(&kv_full[st]);
-                mbar_expect_tx(bar, TB);
-                const CUtensorMap* map = (li & 1) ? &tmV : &tmK;
-                for (int c = 0; c < DCH; ++c)
-                    tma_load_3d(sRing + st * TB + c * kChunkBytes, map, bar, c * 64, (li >> 1) * 128, bk);
+            // K_m and V_m into their own rings, in tile order
+            int issued[2] = {0, 0};   // K and V copies issued
+            bool kv_ok = true;
+            for (int m = 0; m < n_kv && kv_ok; ++m) {
+                for (int which = 0; which < 2 && kv_ok; ++which) {
+                    const int nst = which ? NVR : NKR;
+                    const int st = m % nst;
+                    uint64_t* emp = which ? v_empty : k_empty;
+                    uint64_t* ful = which ? v_full : k_full;
+                    if (!mbar_wait(smem_u32(&emp[st]), ((m / nst) & 1) ^ 1, p.timeout_ns, abort_flag)) {
+                        kv_ok = false;
+                        break;
+                    }
+                    const uint32_t bar = smem_u32(&ful[st]);
+                    mbar_expect_tx(bar, TB);
+                    const uint32_t dst = (which ? sV : sK) + st * TB;
+                    for (int c = 0; c < DCH; ++c)
+                        tma_load_3d(dst + c * kChunkBytes, which ? &tmV : &tmK, bar, c * 64, m * 128, bk);
+                    ++issued[which];
+                }
             }
+            // no copy may still be landing when the CTA exits
             mbar_wait(smem_u32(q_full), 0, p.timeout_ns, nullptr);
-            for (int i = li - 1; i >= 0 && i >= li - NK; --i)
-                mbar_wait(smem_u32(&kv_full[i % NK]), (i / NK) & 1, p.timeout_ns, nullptr);
+            for (int i = issued[0] - 1; i >= 0 && i >= issued[0] - NKR; --i)
+                mbar_wait(smem_u32(&k_full[i % NKR]), (i / NKR) & 1, p.timeout_ns, nullptr);
+            for (int i = issued[1] - 1; i >= 0 && i >= issued[1] - NVR; --i)
+                mbar_wait(smem_u32(&v_full[i % NVR]), (i / NVR) & 1, p.timeout_ns, nullptr);
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
@@ -523,53 +568,73 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const uint32_t idS = idesc_f16(kBF16, 128, 128, false);
             const uint32_t idA = idesc_f16(kBF16, 128, p.d, true);
             const int nk = p.d / 16;
-            const uint64_t aQ = smem_desc_sw128(sQ, 16, 1024);
             const uint64_t adO = smem_desc_sw128(sdO, 16, 1024);
-            const uint64_t bRk = smem_desc_sw128(sRing, 16, 1024);
-            const uint64_t bRm = smem_desc_sw128(sRing, kChunkBytes, 1024);
+            const uint64_t bKk = smem_desc_sw128(sK, 16, 1024);
+            const uint64_t bKm = smem_desc_sw128(sK, kChunkBytes, 1024);
+            const uint64_t bVk = smem_desc_sw128(sV, 16, 1024);
             const auto step = [](int st) { return uint64_t(uint32_t(st) * (TB >> 4)); };
-            const auto full = [&](int li) {
-                return mbar_wait(smem_u32(&kv_full[li % NK]), (li / NK) & 1, p.timeout_ns, abort_flag);
+            const auto kfull = [&](int m) {
+                return mbar_wait(smem_u32(&k_full[m % NKR]), (m / NKR) & 1, p.timeout_ns, abort_flag);
+            };
+            const auto vfull = [&](int m) {
+                return mbar_wait(smem_u32(&v_full[m % NVR]), (m / NVR) & 1, p.timeout_ns, abort_flag);
+            };
+            // S(m) = Q K_m^T with Q from TMEM
+            const auto issue_S = [&](int m) {
+                const uint64_t b0 = bKk + step(m % NKR);
+#pragma unroll
+                for (int kk = 0; kk < 4 * DCH; ++kk) {
+                    if (kk >= nk) break;
+                    const uint64_t off = uint64_t(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+                    mma_ts(tmem, tmem + 448 + kk * 8, b0 + off, idS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(smem_u32(s_full));
+            };
+            const auto issue_dP = [&](int m) {
+                bwd_mma_rows<DCH>(tmem + 128, adO, bVk + step(m % NVR), idS, nk);
+                mma_commit(smem_u32(dp_full));
+                mma_commit(smem_u32(&v_empty[m % NVR]));
             };
             bool ok = mbar_wait(smem_u32(q_full), 0, p.timeout_ns, abort_flag);
-            if (ok) ok = full(0);
+            if (ok) ok = mbar_wait(smem_u32(q_tmem), 0, p.timeout_ns, abort_flag);
+            if (ok) ok = kfull(0);
             if (ok) {
                 tc_fence_after();
-                bwd_mma_rows<DCH>(tmem, aQ, bRk + step(0), idS, nk);
-                mma_commit(smem_u32(s_full));
-                ok = full(1);
+                issue_S(0);
+                ok = vfull(0);
             }
             if (ok) {
                 tc_fence_after();
-                bwd_mma_rows<DCH>(tmem + 128, adO, bRk + step(1 % NK), idS, nk);
-                mma_commit(smem_u32(dp_full));
-                mma_commit(smem_u32(&kv_empty[1 % NK]));
+                issue_dP(0);
             }
             for (int n = 0; n < n_kv && ok; ++n) {
                 const bool more = n + 1 < n_kv;
-                const int liK = 2 * n;
                 ok = mbar_wait(smem_u32(s_read), n & 1, p.timeout_ns, abort_flag);
                 if (!ok) break;
                 if (more) {
-                    ok = full(liK + 2);
+                    ok = kfull(n + 1);
                     if (!ok) break;
                     tc_fence_after();
-                    bwd_mma_rows<DCH>(tmem, aQ, bRk + step((liK + 2) % NK), idS, nk);
-                    mma_commit(smem_u32(s_full));
+                    issue_S(n + 1);
+                }
+                ok = mbar_wait(smem_u32(dp_read), n & 1, p.timeout_ns, abort_flag);
+                if (!ok) break;
+                if (more) {
+                    ok = vfull(n + 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_dP(n + 1);
                 }
                 ok = mbar_wait(smem_u32(ds_ready), n & 1, p.timeout_ns, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                bwd_mma_tmem_a(tmem + 256, tmem + 128, bRm + step(liK % NK), idA, n > 0);
-                mma_commit(smem_u32(&kv_empty[liK % NK]));
-                if (more) {
-                    ok = full(liK + 3);
-                    if (!ok) break;
-                    tc_fence_after();
-                    bwd_mma_rows<DCH>(tmem + 128, adO, bRk + step((liK + 3) % NK), idS, nk);
-                    mma_commit(smem_u32(dp_full));
-                    mma_commit(smem_u32(&kv_empty[(liK + 3) % NK]));
-                }
+                // dS columns 0-127 are TMEM columns 384-447 in order
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + 256, tmem + 384 + kk * 8, bKm + step(n % NKR) + uint64_t((kk * 2048) >> 4),
+                           idA, (n > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(smem_u32(ds_free));
+                mma_commit(smem_u32(&k_empty[n % NKR]));
             }
             mma_commit(smem_u32(acc_done));
             mbar_wait(smem_u32(acc_done), 0, p.timeout_ns, nullptr);
@@ -577,37 +642,60 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     } else if (warp >= 4) {
         // ================================================= elementwise (one query row per thread)
         const int wq = warp & 3;
+        const int half = (warp - 4) >> 2;         // key columns 64*half .. 64*half + 63
         const int row = wq * 32 + lane;
         const uint32_t lane_base = uint32_t(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_base, tdP = tmem + lane_base + 128;
+        const uint32_t tS = tmem + lane_base + 64 * half;
+        const uint32_t tdP = tmem + lane_base + 128 + 64 * half;
+        const uint32_t tdS = tmem + lane_base + 384 + 32 * half;
         const int i = qt * 128 + row;
         const size_t ro = size_t(bh) * p.Tpad + size_t(i);
         const float nl = p.nl[ro];
         const float dd = p.dd[ro];
         const float c2 = p.scale_log2;
-        bool ok = true;
+        // Q row into TMEM (the A operand of S = Q K^T): this half's 64 columns
+        // are one 128-byte row of its swizzled chunk
+        bool ok = mbar_wait(smem_u32(q_full), 0, p.timeout_ns, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            const uint32_t qrow = sQ + uint32_t(half) * kChunkBytes + uint32_t(row >> 3) * 1024 + uint32_t(row & 7) * 128;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                uint32_t w[16];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[4 * u]), "=r"(w[4 * u + 1]), "=r"(w[4 * u + 2]), "=r"(w[4 * u + 3])
+                                 : "r"(qrow + (uint32_t((4 * g + u) ^ (row & 7)) << 4)));
+                tmem_st16(tmem + lane_base + 448 + 32 * half + 16 * g, w);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(q_tmem));
+        }
         for (int n = 0; n < n_kv && ok; ++n) {
             ok = mbar_wait(smem_u32(s_full), n & 1, p.timeout_ns, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            uint32_t r[4][32];
+            uint32_t r[2][32];
             tmem_ld32(tS + 0, r[0]);
             tmem_ld32(tS + 32, r[1]);
-            tmem_ld32(tS + 64, r[2]);
-            tmem_ld32(tS + 96, r[3]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(s_read));
-            // key j = 128 n + c is visible when j < T and (not causal or j <= i)
+            // key j = 128 n + c is visible when j < T and (not causal or j <= i);
+            // `last` is counted from this half's first column
             int last = 127;
             if (n * 128 + 127 >= p.T) last = p.T - 1 - n * 128;
             if (p.causal && n == qt) last = min(last, row);
+            last -= 64 * half;
             const float2 c2v = make_float2(c2, c2);
             const float2 nlv = make_float2(nl, nl);
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch)
+            for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     float2 x = __ffma2_rn(make_float2(__uint_as_float(r[ch][2 * e]),
@@ -623,20 +711,36 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (!ok) break;
             tc_fence_after();
             const float2 ndd = make_float2(-dd, -dd);
+            // dS = P (dP - D) in place of P, then dP's columns are free
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 uint32_t g[32];
                 tmem_ld32(tdP + 32 * ch, g);
                 tmem_wait_ld();
-                uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float2 pp = make_float2(__uint_as_float(r[ch][2 * e]), __uint_as_float(r[ch][2 * e + 1]));
                     const float2 t = __fadd2_rn(make_float2(__uint_as_float(g[2 * e]), __uint_as_float(g[2 * e + 1])), ndd);
                     const float2 ds = __fmul2_rn(pp, t);
-                    pk[e] = pack2<T>(ds.x, ds.y);
+                    r[ch][2 * e] = __float_as_uint(ds.x);
+                    r[ch][2 * e + 1] = __float_as_uint(ds.y);
                 }
-                tmem_st16(tdP + 16 * ch, pk);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(dp_read));
+            // dQ(n-1) must have read the previous dS
+            if (n > 0) ok = mbar_wait(smem_u32(ds_free), (n - 1) & 1, p.timeout_ns, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack2<T>(__uint_as_float(r[ch][2 * e]), __uint_as_float(r[ch][2 * e + 1]));
+                tmem_st16(tdS + 16 * ch, pk);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -649,7 +753,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_after();
             const bool valid = i < p.T;
             const size_t orow = (size_t(bh) * p.T + (valid ? i : 0)) * p.d;
-            bwd_store_row<T>(tmem + lane_base + 256, p.d, p.scale, static_cast<T*>(p.dq) + orow, valid);
+            // the two halves store alternate 16-column pieces of the row
+            bwd_store_row<T>(tmem + lane_base + 256, p.d, p.scale, static_cast<T*>(p.dq) + orow, valid,
+                             16 * half, 32);
         }
     }
 
