@@ -245,12 +245,13 @@ ATTN_API size_t attn_cached_paged_workspace_size(attn_dtype_t dtype, int64_t B, 
  *   [B,H,T,d]: the gradient of the loss with respect to o.
  *   dq [B,H,T,d], dk/dv [B,Hkv,T,d]: overwritten with the gradients; dk and dv
  *   hold the sums over the G = H/Hkv query heads that share each K/V head.
- *   Every tensor row-major and contiguous, 16-byte aligned, one dtype (bf16 or
- *   f16) for all but lse.
+ *   Every tensor row-major and contiguous, 16-byte aligned, one dtype (f32,
+ *   bf16 or f16) for all but lse.
  *   workspace: at least attn_prefill_backward_workspace_size() bytes, 16-byte
  *   aligned; contents on entry irrelevant, scratch afterwards.
- * Supported: bf16/f16 with d a multiple of 16 in [64, 128] (the tensor-core
- * kernels); float32 and other head widths return ATTN_ERR_UNSUPPORTED.
+ * Kernels: bf16/f16 with d a multiple of 16 in [64, 128] on the tensor cores;
+ * float32, and 16-bit head widths outside that set, on CUDA cores in float32
+ * (any d <= 256; larger d returns ATTN_ERR_UNSUPPORTED).
  * Errors as for attn_prefill plus ATTN_ERR_WORKSPACE; checks precede every
  * launch.  An empty problem launches nothing (with H = 0 but B*Hkv*T > 0,
  * dk and dv are set to zero).  Three kernels on `stream`, no allocation, no

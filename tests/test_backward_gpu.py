@@ -11,7 +11,9 @@ the saved O once (so D = dO.O carries one more), and each gradient once on
 output; each of these contributes about u/(2 sqrt 3) relative RMS error, in
 total about 1.2 u = 5e-3 (bf16) normwise.  The bound is 2u normwise (the
 Frobenius norm of the error over that of the gradient, per tensor) and 5u of
-the tensor's largest magnitude for any single element.
+the tensor's largest magnitude for any single element.  float32 runs on the
+CUDA-core kernels with fp32 throughout: u = 5e-6 there (bound 1e-5 normwise,
+as for the float32 forward).
 """
 import math
 
@@ -25,8 +27,8 @@ from transformer_attention_causal_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 
-BF16, F16 = torch.bfloat16, torch.float16
-UNIT = {BF16: 2.0 ** -8, F16: 2.0 ** -11}
+BF16, F16, F32 = torch.bfloat16, torch.float16, torch.float32
+UNIT = {BF16: 2.0 ** -8, F16: 2.0 ** -11, F32: 5e-6}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -75,6 +77,12 @@ CASES = [
     (F16, 2, 2, 1, 100, 128, True),      # one partial tile
     (BF16, 1, 6, 3, 1000, 128, True),    # many tiles
     (F16, 1, 2, 2, 700, 112, False),     # full attention, d = 112
+    # CUDA-core kernels: float32, and 16-bit head sizes outside the tensor-core set
+    (F32, 1, 4, 2, 130, 64, True),
+    (F32, 2, 2, 1, 77, 40, False),
+    (F32, 1, 2, 2, 200, 256, True),
+    (BF16, 1, 2, 2, 150, 48, True),
+    (F16, 1, 4, 1, 100, 200, True),
 ]
 
 

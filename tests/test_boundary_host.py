@@ -224,16 +224,19 @@ def test_backward_rejects_invalid_arguments(lib, kwargs):
     assert backward(lib, **kwargs) == INVALID
 
 
-@pytest.mark.parametrize("kwargs", [dict(dt=F32), dict(d=48), dict(d=136), dict(d=72)])
-def test_backward_rejects_unsupported_shapes(lib, kwargs):
-    assert backward(lib, **kwargs) == UNSUPPORTED
+def test_backward_rejects_unsupported_shapes(lib):
+    # float32 and 16-bit head sizes off the tensor-core set run on CUDA cores;
+    # only d > 256 is refused
+    assert backward(lib, d=264) == UNSUPPORTED
+    for kwargs in (dict(dt=F32), dict(d=48), dict(d=136), dict(d=72), dict(dt=F32, d=256)):
+        assert backward(lib, ws=None, ws_bytes=0, **kwargs) == WORKSPACE
 
 
 def test_backward_workspace(lib):
     # two float32 row statistics per padded query row: 300 rows pad to 384
     need = lib.attn_prefill_backward_workspace_size(BF16, 2, 4, 2, 300, 128)
     assert need == 2 * 2 * 4 * 384 * 4
-    assert lib.attn_prefill_backward_workspace_size(F32, 2, 4, 2, 300, 128) == 0
+    assert lib.attn_prefill_backward_workspace_size(F32, 2, 4, 2, 300, 128) == need
     assert lib.attn_prefill_backward_workspace_size(BF16, 2, 4, 2, 0, 128) == 0
     assert backward(lib, B=2, ws=FAKE, ws_bytes=need - 1) == WORKSPACE
     assert backward(lib, B=2, ws=None, ws_bytes=need) == WORKSPACE

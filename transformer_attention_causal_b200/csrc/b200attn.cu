@@ -17,6 +17,7 @@
 #include "prefill_backward.cuh"
 #include "prefill_tcgen05.cuh"
 #include "simt_attn.cuh"
+#include "simt_backward.cuh"
 
 using namespace b200attn;
 
@@ -479,17 +480,36 @@ attn_status_t launch_append(AppendParams& ap, cudaStream_t stream) {
 
 namespace {
 
-// Shapes the tensor-core backward kernels take.
+// The tensor-core backward kernels take 16-bit inputs with d a multiple of
+// 16 in [64, 128]; everything else up to d = 256 runs on CUDA cores.
+bool backward_on_tensor_cores(const Problem& pb) {
+    return pb.dt != ATTN_F32 && pb.d % 16 == 0 && pb.d >= 64 && pb.d <= 128;
+}
+
 attn_status_t check_backward(const Problem& pb) {
     attn_status_t st = check_shape(pb);
     if (st != ATTN_OK || empty_problem(pb)) return st;
-    if (pb.dt == ATTN_F32) return ATTN_ERR_UNSUPPORTED;
-    if (pb.d % 16 != 0 || pb.d < 64 || pb.d > 128) return ATTN_ERR_UNSUPPORTED;
     const int64_t n_t = (pb.Tq + 127) / 128;
+    const int64_t rows = std::max(pb.B * pb.H, pb.B * pb.Hkv) * n_t * 128;
     if (n_t * pb.B * pb.H >= (int64_t(1) << 31) || pb.Tq >= (int64_t(1) << 30) ||
-        pb.S_cap * pb.d * 2 >= (int64_t(1) << 40))
+        rows / kSimtBwdWarps >= (int64_t(1) << 31) || pb.S_cap * pb.d * 2 >= (int64_t(1) << 40))
         return ATTN_ERR_UNSUPPORTED;
     return ATTN_OK;
+}
+
+template <typename T>
+attn_status_t launch_backward_simt(BwdParams& bp, const void* q, const void* k, const void* v,
+                                   cudaStream_t stream) {
+    const SimtBwdPtrs in{q, k, v};
+    const auto blocks = [](int64_t rows) { return unsigned((rows + kSimtBwdWarps - 1) / kSimtBwdWarps); };
+    simt_bwd_preprocess_kernel<T><<<blocks(int64_t(bp.B) * bp.H * bp.Tpad), kSimtBwdWarps * 32, 0,
+                                    stream>>>(bp);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
+    simt_bwd_dkdv_kernel<T><<<blocks(int64_t(bp.B) * bp.Hkv * bp.T), kSimtBwdWarps * 32, 0, stream>>>(
+        bp, in);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
+    simt_bwd_dq_kernel<T><<<blocks(int64_t(bp.B) * bp.H * bp.T), kSimtBwdWarps * 32, 0, stream>>>(bp, in);
+    return launch_status();
 }
 
 size_t backward_ws_bytes(const Problem& pb) {
@@ -633,6 +653,11 @@ attn_status_t attn_prefill_backward(const void* q, const void* k, const void* v,
     bp.scale_log2 = scale * 1.4426950408889634f;
     bp.timeout_ns = g_timeout_ns.load();
     const bool bf16 = dtype == ATTN_BF16;
+    if (!backward_on_tensor_cores(pb)) {
+        if (dtype == ATTN_F32) return launch_backward_simt<float>(bp, q, k, v, s);
+        return bf16 ? launch_backward_simt<__nv_bfloat16>(bp, q, k, v, s)
+                    : launch_backward_simt<__half>(bp, q, k, v, s);
+    }
     if (d <= 64)
         return bf16 ? launch_backward<__nv_bfloat16, 1>(pb, bp, q, k, v, dout, s)
                     : launch_backward<__half, 1>(pb, bp, q, k, v, dout, s);
