@@ -194,9 +194,12 @@ def test_paged_rejects_invalid_arguments(lib, kwargs):
 
 
 def test_paged_limits(lib):
-    assert paged(lib, dt=F32) == UNSUPPORTED            # float32 has no split-KV kernel
-    assert paged(lib, H=32, Hkv=1, Tnew=1) == UNSUPPORTED   # 32 rows per K/V head
-    assert paged(lib, d=80) == UNSUPPORTED
+    assert paged(lib, dt=F32) == UNSUPPORTED            # float32 has no paged kernel
+    # many rows per K/V head go to the tensor-core prefill, which takes d in
+    # [64, 128]; other head sizes have no paged kernel
+    assert paged(lib, H=32, Hkv=1, Tnew=1, d=48) == UNSUPPORTED
+    assert paged(lib, H=32, Hkv=1, Tnew=1, d=256) == UNSUPPORTED
+    assert paged(lib, d=72) == UNSUPPORTED
     # empty problems launch nothing
     assert paged(lib, q=None, kp=None, vp=None, o=None, table=None, lens=None, B=0) == 0
     # a split plan needs workspace

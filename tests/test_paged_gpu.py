@@ -80,6 +80,13 @@ CASES = [
     (2, 8, 1, 1, 64, [333, 64], 8, BF16),              # MQA, d = 64, the smallest pages
     (2, 4, 4, 2, 256, [900, 129], 32, F16),            # d = 256
     (4, 8, 8, 1, 128, [1, 5, 128, 129], 128, BF16),    # lengths at page edges, a single token
+    # chunked prefill (many new rows per K/V head): the tensor-core kernel
+    # copying whole pages, one to sixteen copies per 128-key tile
+    (2, 8, 1, 200, 128, [1000, 450], 64, F16),         # MQA, two pages per tile
+    (2, 16, 4, 300, 128, [800, 300], 128, BF16),       # a page per tile; a sequence of only new tokens
+    (1, 8, 2, 129, 64, [2000], 256, BF16),             # pages longer than a tile, d = 64
+    (2, 4, 4, 64, 80, [129, 1000], 16, F16),           # MHA, d = 80
+    (3, 8, 2, 100, 96, [100, 357, 1024], 8, BF16),     # the smallest pages
 ]
 
 
@@ -129,6 +136,14 @@ def test_out_of_range_entries_are_reported_not_followed(what):
         kv_lens[0] = 250
         bound = 200
     run_gpu(q, kp, vp, table, kv_lens, 0.1, max_kv_len=bound)
+    assert attn.device_status() == DEVICE_INDEX
+    assert attn.device_status() == 0
+
+
+def test_out_of_range_page_in_chunked_prefill_is_reported():
+    q, kp, vp, table, kv_lens = make_paged(2, 8, 2, 150, 128, [300, 200], 16, BF16, seed=6)
+    table[1, 3] = kp.shape[0] + 5
+    run_gpu(q, kp, vp, table, kv_lens, 0.1)
     assert attn.device_status() == DEVICE_INDEX
     assert attn.device_status() == 0
 

@@ -187,12 +187,13 @@ attn_status_t get_encoder() {
     return g_encode ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// [nslices, rows (pitch row_pitch), d] 16-bit tensor, box of 64 columns x 128 rows.
+// [nslices, rows (pitch row_pitch), d] 16-bit tensor, box of 64 columns x
+// box_rows rows (128 unless a paged pool's pages are smaller).
 attn_status_t encode_rows(CUtensorMap* map, const void* ptr, attn_dtype_t dt, int64_t d,
-                          int64_t rows, int64_t row_pitch, int64_t nslices) {
+                          int64_t rows, int64_t row_pitch, int64_t nslices, uint32_t box_rows = 128) {
     const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(nslices)};
     const cuuint64_t strides[2] = {cuuint64_t(d * 2), cuuint64_t(row_pitch * d * 2)};
-    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t box[3] = {64, box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapDataType ty =
         dt == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -365,12 +366,12 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
     }
 }
 
-template <typename T, int DCH, bool WINDOW>
+template <typename T, int DCH, bool WINDOW, bool PAGED = false>
 attn_status_t launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk,
                                     const CUtensorMap& mv, const PrefillParams& pp, int64_t grid,
                                     cudaStream_t stream) {
     constexpr size_t smem = prefill_smem_bytes<DCH>();
-    auto kern = prefill_tcgen05_kernel<T, DCH, WINDOW>;
+    auto kern = prefill_tcgen05_kernel<T, DCH, WINDOW, PAGED>;
     static std::once_flag once[8];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -391,7 +392,7 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
         encode_rows(&mk, k, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK ||
         encode_rows(&mv, v, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK)
         return ATTN_ERR_CUDA;
-    PrefillParams pp;
+    PrefillParams pp{};
     pp.o = o; pp.lse = lse;
     pp.B = int(pb.B); pp.H = int(pb.H); pp.Hkv = int(pb.Hkv); pp.G = int(pb.H / pb.Hkv);
     pp.Tq = int(pb.Tq); pp.S = pb.S; pp.start_pos = pb.start_pos; pp.d = int(pb.d);
@@ -407,6 +408,41 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
     const int64_t grid = std::min<int64_t>(units, sm_count());
     return pb.window > 0 ? launch_prefill_kernel<T, DCH, true>(mq, mk, mv, pp, grid, stream)
                          : launch_prefill_kernel<T, DCH, false>(mq, mk, mv, pp, grid, stream);
+}
+
+// The tensor-core prefill over a paged cache (chunked prefill): K/V maps over
+// the pools [num_pages * Hkv, P, d] with boxes of min(P, 128) rows.
+template <typename T, int DCH>
+attn_status_t launch_prefill_paged(const Problem& pb, const Plan& pl, const void* q, const void* kp,
+                                   const void* vp, void* o, float* lse, float scale,
+                                   const PagedKV& pk, int64_t page_size, cudaStream_t stream) {
+    if (get_encoder() != ATTN_OK) return ATTN_ERR_CUDA;
+    CUtensorMap mq, mk, mv;
+    const uint32_t rows = uint32_t(std::min<int64_t>(page_size, 128));
+    if (encode_rows(&mq, q, pb.dt, pb.d, pb.Tq, pb.Tq, pb.B * pb.H) != ATTN_OK ||
+        encode_rows(&mk, kp, pb.dt, pb.d, page_size, page_size, pk.num_pages * pb.Hkv, rows) != ATTN_OK ||
+        encode_rows(&mv, vp, pb.dt, pb.d, page_size, page_size, pk.num_pages * pb.Hkv, rows) != ATTN_OK)
+        return ATTN_ERR_CUDA;
+    PrefillParams pp{};
+    pp.o = o; pp.lse = lse;
+    pp.B = int(pb.B); pp.H = int(pb.H); pp.Hkv = int(pb.Hkv); pp.G = int(pb.H / pb.Hkv);
+    pp.Tq = int(pb.Tq); pp.S = pb.S; pp.start_pos = pb.start_pos; pp.d = int(pb.d);
+    pp.causal = 1; pp.pair_mode = pl.pair_mode; pp.n_qb = pl.n_qb;
+    pp.window = 0;
+    pp.units_per_level = pl.units_per_level;
+    pp.n_levels = pl.n_levels;
+    pp.scale_log2 = scale * 1.4426950408889634f;
+    pp.timeout_ns = g_timeout_ns.load();
+    pp.test_flags = g_test_flags.load();
+    pp.page_table = pk.page_table;
+    pp.kv_lens = pk.kv_lens;
+    pp.max_pages = pk.max_pages;
+    pp.num_pages = pk.num_pages;
+    pp.max_kv_len = pb.S;
+    pp.page_shift = pk.page_shift;
+    const int64_t units = int64_t(pl.units_per_level) * pl.n_levels;
+    const int64_t grid = std::min<int64_t>(units, sm_count());
+    return launch_prefill_kernel<T, DCH, false, true>(mq, mk, mv, pp, grid, stream);
 }
 
 template <typename T>
@@ -719,10 +755,11 @@ attn_status_t attn_cached_paged(const void* q, const void* k_pages, const void* 
     Plan pl;
     attn_status_t st = make_plan(pb, pl);
     if (st != ATTN_OK) return st;
-    if (pl.kernel != ATTN_KERNEL_SPLITKV) return ATTN_ERR_UNSUPPORTED;
+    if (pl.kernel != ATTN_KERNEL_SPLITKV && pl.kernel != ATTN_KERNEL_TCGEN05) return ATTN_ERR_UNSUPPORTED;
     st = check_pointers(pb, q, k_pages, v_pages, o, lse);
     if (st != ATTN_OK) return st;
-    if (num_pages * Hkv * page_size * d > (int64_t(1) << 46)) return ATTN_ERR_UNSUPPORTED;
+    if (num_pages * Hkv * page_size * d > (int64_t(1) << 46) || num_pages * Hkv >= (int64_t(1) << 31))
+        return ATTN_ERR_UNSUPPORTED;
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return ATTN_ERR_WORKSPACE;
         if (!aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
@@ -734,6 +771,18 @@ attn_status_t attn_cached_paged(const void* q, const void* k_pages, const void* 
     pk.num_pages = num_pages;
     while ((int64_t(1) << pk.page_shift) < page_size) ++pk.page_shift;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pl.kernel == ATTN_KERNEL_TCGEN05) {
+        const bool bf16 = dtype == ATTN_BF16;
+        if (pl.dch == 1)
+            return bf16 ? launch_prefill_paged<__nv_bfloat16, 1>(pb, pl, q, k_pages, v_pages, o, lse, scale, pk,
+                                                                 page_size, s)
+                        : launch_prefill_paged<__half, 1>(pb, pl, q, k_pages, v_pages, o, lse, scale, pk,
+                                                          page_size, s);
+        return bf16 ? launch_prefill_paged<__nv_bfloat16, 2>(pb, pl, q, k_pages, v_pages, o, lse, scale, pk,
+                                                             page_size, s)
+                    : launch_prefill_paged<__half, 2>(pb, pl, q, k_pages, v_pages, o, lse, scale, pk,
+                                                      page_size, s);
+    }
     if (dtype == ATTN_BF16)
         return run_decode<__nv_bfloat16>(pb, pl, q, k_pages, v_pages, o, lse, scale, workspace, s, &pk);
     return run_decode<__half>(pb, pl, q, k_pages, v_pages, o, lse, scale, workspace, s, &pk);

@@ -60,7 +60,6 @@ struct DecodeParams {
     int64_t max_pages, num_pages;
 };
 
-constexpr unsigned kStatusBadIndex = 6u;   // a page table or length entry out of range
 
 // Positions of a unit's rows: its new tokens start at `start_pos` and the
 // visible keys end at `kv_end`.  For a paged cache both come from the

@@ -59,6 +59,13 @@ struct PrefillParams {
     float scale_log2;    // scale * log2(e)
     uint64_t timeout_ns;
     uint32_t test_flags;  // kTestSkipLoads: issue no K/V copies (timeout-path tests)
+    // paged K/V (the PAGED kernel): pools [num_pages, Hkv, 2^page_shift, d];
+    // key j of sequence b is row j % P of page page_table[b * max_pages + j / P];
+    // sequence b holds kv_lens[b] keys, its Tq new queries being the last ones
+    const int32_t* page_table;
+    const int32_t* kv_lens;
+    int64_t max_pages, num_pages, max_kv_len;
+    int page_shift;
 };
 
 constexpr int kPfThreads = 384;  // 12 warps
@@ -168,26 +175,30 @@ constexpr size_t prefill_smem_bytes() {
 // n_full) are visible to every row of it, the others are masked.
 struct SlotInfo {
     int h, q0, n_lo, n_kv, n_full_lo, n_full;
+    int64_t S, start;   // keys of the slot's sequence, position of its query row 0
 };
 
 template <bool WINDOW>
-__device__ __forceinline__ SlotInfo prefill_slot(const PrefillParams& p, int h, int qb) {
+__device__ __forceinline__ SlotInfo prefill_slot(const PrefillParams& p, int h, int qb, int64_t S,
+                                                 int64_t start) {
     SlotInfo s;
     s.h = h;
     s.q0 = qb * 128;
+    s.S = S;
+    s.start = start;
     if (s.q0 >= p.Tq) {
         s.n_lo = s.n_kv = s.n_full_lo = s.n_full = 0;
         return s;
     }
     const int64_t qlast = min64(s.q0 + 127, p.Tq - 1);
-    const int64_t kv_end = p.causal ? min64(p.S, p.start_pos + qlast + 1) : p.S;
+    const int64_t kv_end = p.causal ? min64(S, start + qlast + 1) : S;
     s.n_kv = int((kv_end + 127) / 128);
-    const int64_t full_c = p.causal ? (p.start_pos + s.q0 + 1) / 128 : (p.S / 128);
-    s.n_full = int(min64(full_c, p.S / 128));
+    const int64_t full_c = p.causal ? (start + s.q0 + 1) / 128 : (S / 128);
+    s.n_full = int(min64(full_c, S / 128));
     s.n_lo = s.n_full_lo = 0;
     if (WINDOW) {
-        const int64_t first = max64(0, p.start_pos + s.q0 - p.window + 1);   // lowest key seen
-        const int64_t all_lo = max64(0, p.start_pos + qlast - p.window + 1);  // every row sees from here
+        const int64_t first = max64(0, start + s.q0 - p.window + 1);   // lowest key seen
+        const int64_t all_lo = max64(0, start + qlast - p.window + 1);  // every row sees from here
         s.n_lo = int(first / 128);
         s.n_full_lo = int((all_lo + 127) / 128);
     }
@@ -230,27 +241,66 @@ __device__ __forceinline__ void issue_PV(uint64_t dV0, uint32_t tmem, uint32_t i
 
 // The unit of work a CTA does at pass `unit`: its batch entry, K/V head and
 // two slots (heaviest first: the longest causal row range first).
-template <bool WINDOW>
+template <bool WINDOW, bool PAGED>
 __device__ __forceinline__ void prefill_unit(const PrefillParams& p, int unit, int& b, int& kvh,
                                              SlotInfo (&slot)[2]) {
     const int level = unit / p.units_per_level;
     const int rem = unit % p.units_per_level;
+    int h0, h1, qb0, qb1;
     if (p.pair_mode == 0) {
         const int half = p.G / 2;
-        const int qb = p.n_qb - 1 - level;
         b = rem / (p.Hkv * half);
         const int r2 = rem % (p.Hkv * half);
         kvh = r2 / half;
-        const int h0 = kvh * p.G + 2 * (r2 % half);
-        slot[0] = prefill_slot<WINDOW>(p, h0, qb);
-        slot[1] = prefill_slot<WINDOW>(p, h0 + 1, qb);
+        h0 = kvh * p.G + 2 * (r2 % half);
+        h1 = h0 + 1;
+        qb0 = qb1 = p.n_qb - 1 - level;
     } else {
         const int qbp = p.n_levels - 1 - level;
         b = rem / p.H;
-        const int h = rem % p.H;
-        kvh = h / p.G;
-        slot[0] = prefill_slot<WINDOW>(p, h, 2 * qbp);
-        slot[1] = prefill_slot<WINDOW>(p, h, 2 * qbp + 1);
+        h0 = h1 = rem % p.H;
+        kvh = h0 / p.G;
+        qb0 = 2 * qbp;
+        qb1 = qb0 + 1;
+    }
+    int64_t S = p.S, start = p.start_pos;
+    if (PAGED) {
+        // a length outside [Tq, max_kv_len] is reported and clamped
+        int64_t L = p.kv_lens[b];
+        if (L < p.Tq || L > p.max_kv_len) {
+            atomicCAS(&g_device_status, 0u, kStatusBadIndex);
+            L = max64(int64_t(p.Tq), min64(L, p.max_kv_len));
+        }
+        S = L;
+        start = L - p.Tq;
+    }
+    slot[0] = prefill_slot<WINDOW>(p, h0, qb0, S, start);
+    slot[1] = prefill_slot<WINDOW>(p, h1, qb1, S, start);
+}
+
+// K or V tile n of sequence b, head kvh, from a paged pool: one TMA copy per
+// page the tile spans (min(P, 128) rows each).  Rows past the sequence's end,
+// and pages whose id is out of range (reported), are read at an out-of-range
+// coordinate, which TMA fills with zeros while still counting the bytes.
+template <int DCH>
+__device__ __forceinline__ void load_kv_paged(const PrefillParams& p, uint32_t dst, const CUtensorMap* map,
+                                              uint32_t bar, int n, int b, int kvh, int64_t L) {
+    const int rows = min(1 << p.page_shift, 128);
+    for (int sub = 0; sub < 128 / rows; ++sub) {
+        const int64_t tok = int64_t(n) * 128 + int64_t(sub) * rows;
+        int64_t z = p.num_pages * p.Hkv;   // past the pools: zero fill
+        int y = 0;
+        if (tok < L) {
+            const int32_t phys = p.page_table[int64_t(b) * p.max_pages + (tok >> p.page_shift)];
+            if (phys < 0 || phys >= p.num_pages) {
+                atomicCAS(&g_device_status, 0u, kStatusBadIndex);
+            } else {
+                z = int64_t(phys) * p.Hkv + kvh;
+                y = int(tok & ((int64_t(1) << p.page_shift) - 1));
+            }
+        }
+        for (int c = 0; c < DCH; ++c)
+            tma_load_3d(dst + c * kChunkBytes + uint32_t(sub * rows) * 128u, map, bar, c * 64, y, int32_t(z));
     }
 }
 
@@ -261,7 +311,7 @@ __device__ __forceinline__ int prefill_pass_unit(int k) {
                         : (k + 1) * int(gridDim.x) - 1 - int(blockIdx.x);
 }
 
-template <typename T, int DCH, bool WINDOW>
+template <typename T, int DCH, bool WINDOW, bool PAGED>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -334,7 +384,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (unit >= n_units) break;
                 int b, kvh;
                 SlotInfo slot[2];
-                prefill_unit<WINDOW>(p, unit, b, kvh, slot);
+                prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
                 const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                 const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                  : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
@@ -366,9 +416,13 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const uint32_t bar = smem_u32(&kv_full[st]);
                     mbar_expect_tx(bar, DCH * kChunkBytes);
                     const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
-                    for (int c = 0; c < DCH; ++c)
-                        tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64,
-                                    (nmin + (i >> 1)) * 128, zkv);
+                    if (PAGED)
+                        load_kv_paged<DCH>(p, sRing + st * DCH * kChunkBytes, map, bar, nmin + (i >> 1), b,
+                                           kvh, slot[0].S);
+                    else
+                        for (int c = 0; c < DCH; ++c)
+                            tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64,
+                                        (nmin + (i >> 1)) * 128, zkv);
                 }
             }
             // no copy may still be landing in shared memory when the CTA exits
@@ -396,7 +450,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (unit >= n_units) break;
                 int b, kvh;
                 SlotInfo slot[2];
-                prefill_unit<WINDOW>(p, unit, b, kvh, slot);
+                prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
                 const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                 const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                  : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
@@ -494,10 +548,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (unit >= n_units) break;
             int b, kvh;
             SlotInfo slot[2];
-            prefill_unit<WINDOW>(p, unit, b, kvh, slot);
+            prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
             const SlotInfo sl = slot[s];
             if (sl.n_kv == 0) continue;
-            const int64_t qpos = p.start_pos + sl.q0 + row;
+            const int64_t qpos = sl.start + sl.q0 + row;
             float m_run = -INFINITY, l = 0.f;
             for (int n = sl.n_lo; n < sl.n_kv; ++n) {
                 ok = mbar_wait(smem_u32(&s_full[s]), scount & 1, p.timeout_ns, abort_flag);
@@ -516,7 +570,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const bool masked = n >= sl.n_full || (WINDOW && n < sl.n_full_lo);
                 if (masked) {
                     int64_t lim = p.causal ? qpos - int64_t(n) * 128 : 127;
-                    lim = min64(lim, p.S - 1 - int64_t(n) * 128);
+                    lim = min64(lim, sl.S - 1 - int64_t(n) * 128);
                     const int li = int(max64(-1, min64(127, lim)));
                     mask_chunk(r0, li);
                     mask_chunk(r1, li - 32);

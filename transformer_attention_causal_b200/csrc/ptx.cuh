@@ -15,6 +15,7 @@ namespace b200attn {
 __device__ unsigned int g_device_status;
 
 constexpr unsigned kStatusTimeout = 5u;  // == ATTN_ERR_DEVICE_TIMEOUT
+constexpr unsigned kStatusBadIndex = 6u; // == ATTN_ERR_DEVICE_INDEX: a page table or length entry out of range
 
 // Test hook (attn_test_set_flags): producers issue no K/V copies, so every
 // consumer's bounded wait runs out and the timeout path is exercised.
