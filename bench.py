@@ -352,24 +352,31 @@ class Case:
         if self.kernel == "splitkv" and self.ws is not None:
             self.launches = 2
 
-    def call(self):
+    def call(self, bufs=None, stream=None):
+        """One library call on (inputs, outputs) = bufs (default: the case's
+        own device buffers), enqueued on `stream` (default: the current one)."""
         w = self.w
+        dev_in, dev_out = bufs if bufs is not None else (self.dev_in, self.dev_out)
         if w["kind"] == "append":
-            self.attn.kv_append_rope(*self.dev_in, *self.dev_out, start_pos=w["start"],
-                                     rope_base=w["base"])
+            self.attn.kv_append_rope(*dev_in, *dev_out, start_pos=w["start"], rope_base=w["base"],
+                                     stream=stream)
         elif w["kind"] == "backward":
-            dq, dk, dv = self.dev_out
-            self.attn.prefill_backward(*self.dev_in, scale=self.scale, causal=True, dq=dq, dk=dk,
-                                       dv=dv, workspace=self.ws)
+            dq, dk, dv = dev_out
+            self.attn.prefill_backward(*dev_in, scale=self.scale, causal=True, dq=dq, dk=dk, dv=dv,
+                                       workspace=self.ws, stream=stream)
         elif w["kind"] == "prefill":
-            self.attn.prefill(self.q, self.k, self.v, scale=self.scale, causal=True, out=self.out,
-                              window=w.get("window", 0))
+            q, k, v = dev_in
+            self.attn.prefill(q, k, v, scale=self.scale, causal=True, out=dev_out[0],
+                              window=w.get("window", 0), stream=stream)
         elif w["kind"] == "paged":
-            self.attn.cached_paged(self.q, self.k, self.v, self.table, self.lens, max_kv_len=w["S"],
-                                   scale=self.scale, out=self.out, workspace=self.ws)
+            q, k, v = dev_in
+            self.attn.cached_paged(q, k, v, self.table, self.lens, max_kv_len=w["S"],
+                                   scale=self.scale, out=dev_out[0], workspace=self.ws,
+                                   stream=stream)
         else:
-            self.attn.cached(self.q, self.k, self.v, start_pos=w["start"], scale=self.scale,
-                             out=self.out, workspace=self.ws)
+            q, k, v = dev_in
+            self.attn.cached(q, k, v, start_pos=w["start"], scale=self.scale, out=dev_out[0],
+                             workspace=self.ws, stream=stream)
 
 
 def time_device(case, steps, warmup, dist_ctx):
@@ -400,24 +407,54 @@ def time_device(case, steps, warmup, dist_ctx):
 
 def time_e2e(case, steps, warmup, dist_ctx):
     """Per-step time (ms) with the inputs copied host -> device from pinned
-    memory and the output copied back, every step."""
-    def step():
-        for dev, host in zip(case.dev_in, case.host):
-            dev.copy_(host, non_blocking=True)
-        case.call()
-        for host, dev in zip(case.host_out, case.dev_out):
-            host.copy_(dev, non_blocking=True)
+    memory and the output copied back, every step, through the public API.
 
-    for _ in range(warmup):
-        step()
+    Steps are pipelined over two device buffer sets and three streams, the way
+    a serving loop would run them: step k's host -> device copy overlaps step
+    k-1's call and step k-2's device -> host copy.  Every step still moves all
+    of its bytes; events order each buffer's reuse."""
+    sets = [(case.dev_in, case.dev_out),
+            ([torch.empty_like(t) for t in case.dev_in], [torch.empty_like(t) for t in case.dev_out])]
+    s_h2d, s_call, s_d2h = (torch.cuda.Stream(device=case.device) for _ in range(3))
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    h2d_done, call_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    used = [False, False]
+
+    def step(k):
+        slot = k & 1
+        dev_in, dev_out = sets[slot]
+        with torch.cuda.stream(s_h2d):
+            if used[slot]:
+                s_h2d.wait_event(call_done[slot])     # the call of step k-2 has read dev_in
+            for dev, host in zip(dev_in, case.host):
+                dev.copy_(host, non_blocking=True)
+            h2d_done[slot].record(s_h2d)
+        s_call.wait_event(h2d_done[slot])
+        if used[slot]:
+            s_call.wait_event(d2h_done[slot])         # step k-2's result has left dev_out
+        case.call((dev_in, dev_out), stream=s_call)
+        call_done[slot].record(s_call)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(call_done[slot])
+            for host, dev in zip(case.host_out, dev_out):
+                host.copy_(dev, non_blocking=True)
+            d2h_done[slot].record(s_d2h)
+        used[slot] = True
+
+    for k in range(warmup):
+        step(k)
     b0 = torch.cuda.Event(enable_timing=True)
     b1 = torch.cuda.Event(enable_timing=True)
     dist_ctx.barrier()
     torch.cuda.synchronize()
-    b0.record()
-    for _ in range(steps):
-        step()
-    b1.record()
+    b0.record(s_h2d)
+    s_call.wait_stream(s_h2d)
+    s_d2h.wait_stream(s_h2d)
+    for k in range(warmup, warmup + steps):
+        step(k)
+    s_d2h.wait_stream(s_call)
+    s_d2h.wait_stream(s_h2d)
+    b1.record(s_d2h)
     torch.cuda.synchronize()
     dist_ctx.barrier()
     h2d = sum(t.numel() * t.element_size() for t in case.host)
