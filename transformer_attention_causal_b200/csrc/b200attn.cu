@@ -400,7 +400,8 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
     pp.window = pb.window;
     pp.units_per_level = pl.units_per_level;
     pp.n_levels = pl.n_levels;
-    pp.scale_log2 = scale * 1.4426950408889634f;
+    pp.scale_log2 = scale == 0.f ? 1.f : std::fabs(scale) * 1.4426950408889634f;
+    pp.score_mode = scale > 0.f ? 0 : (scale < 0.f ? 1 : 2);
     pp.timeout_ns = g_timeout_ns.load();
     pp.test_flags = g_test_flags.load();
     // persistent CTAs, one per SM (the kernel deals the units out itself)
@@ -431,7 +432,8 @@ attn_status_t launch_prefill_paged(const Problem& pb, const Plan& pl, const void
     pp.window = 0;
     pp.units_per_level = pl.units_per_level;
     pp.n_levels = pl.n_levels;
-    pp.scale_log2 = scale * 1.4426950408889634f;
+    pp.scale_log2 = scale == 0.f ? 1.f : std::fabs(scale) * 1.4426950408889634f;
+    pp.score_mode = scale > 0.f ? 0 : (scale < 0.f ? 1 : 2);
     pp.timeout_ns = g_timeout_ns.load();
     pp.test_flags = g_test_flags.load();
     pp.page_table = pk.page_table;

@@ -56,7 +56,8 @@ struct PrefillParams {
     int n_qb;            // ceil(Tq / 128)
     int units_per_level;
     int n_levels;        // units = units_per_level * n_levels, heaviest level first
-    float scale_log2;    // scale * log2(e)
+    float scale_log2;    // |scale| * log2(e) (1 when scale = 0)
+    int score_mode;      // 0: scale > 0; 1: scale < 0 (scores negated); 2: scale = 0 (scores zeroed)
     uint64_t timeout_ns;
     uint32_t test_flags;  // kTestSkipLoads: issue no K/V copies (timeout-path tests)
     // paged K/V (the PAGED kernel): pools [num_pages, Hkv, 2^page_shift, d];
@@ -567,6 +568,19 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tmem_ld32(tS + 64, r2);
                 tmem_ld32(tS + 96, r3);
                 tmem_wait_ld();
+                if (p.score_mode != 0) {
+                    // scale < 0 is attention on -S with |scale|; scale = 0 weighs
+                    // every visible key alike (the mask below still applies)
+                    const uint32_t flip = p.score_mode == 1 ? 0x80000000u : 0u;
+                    const uint32_t keep = p.score_mode == 1 ? 0xffffffffu : 0u;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        r0[e] = (r0[e] & keep) ^ flip;
+                        r1[e] = (r1[e] & keep) ^ flip;
+                        r2[e] = (r2[e] & keep) ^ flip;
+                        r3[e] = (r3[e] & keep) ^ flip;
+                    }
+                }
                 const bool masked = n >= sl.n_full || (WINDOW && n < sl.n_full_lo);
                 if (masked) {
                     int64_t lim = p.causal ? qpos - int64_t(n) * 128 : 127;
