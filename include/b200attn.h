@@ -269,6 +269,20 @@ ATTN_API attn_status_t attn_prefill_backward(const void* q, const void* k, const
                                              int64_t B, int64_t H, int64_t Hkv, int64_t T,
                                              int64_t d, float scale, int causal, void* workspace,
                                              size_t workspace_bytes, void* stream);
+/* The backward pass of local attention (attn_prefill_local's forward): row i
+ * reads keys i - window < j <= i, so gradients flow only through those scores
+ * ("Multi-query attention, annotated" §4.1; "Causal Multi-Head
+ * Self-Attention", Causal mask: a masked score carries zero gradient).
+ * Arguments, kernels, workspace and errors as for attn_prefill_backward
+ * (always causal); window = 0, or a window of at least T, is plain causal
+ * attention; window < 0 returns ATTN_ERR_INVALID_ARG. */
+ATTN_API attn_status_t attn_prefill_backward_local(const void* q, const void* k, const void* v,
+                                                   const void* o, const float* lse, const void* dout,
+                                                   void* dq, void* dk, void* dv, attn_dtype_t dtype,
+                                                   int64_t B, int64_t H, int64_t Hkv, int64_t T,
+                                                   int64_t d, float scale, int64_t window,
+                                                   void* workspace, size_t workspace_bytes,
+                                                   void* stream);
 
 /* Bytes of workspace attn_cached needs for this problem (0 if none).  Pure
  * host arithmetic; valid without a GPU.  Returns 0 for arguments that

@@ -98,6 +98,32 @@ def test_backward_matches_oracle(case):
         check(name, g, r, dtype)
 
 
+WINDOWED = [
+    # dtype, B, H, Hkv, T, d, window
+    (BF16, 1, 4, 2, 500, 128, 32),       # the pages' window of 32
+    (F16, 1, 2, 1, 700, 64, 300),        # a window spanning several tiles
+    (BF16, 1, 2, 2, 1000, 80, 128),      # window = one tile
+    (F32, 1, 2, 1, 150, 64, 20),         # CUDA-core kernels
+    (BF16, 1, 2, 2, 200, 48, 50),
+]
+
+
+@pytest.mark.parametrize("case", WINDOWED, ids=lambda c: "-".join(map(str, c)))
+def test_windowed_backward_matches_oracle(case):
+    dtype, B, H, Hkv, T, d, w = case
+    q, k, v = inputs.qkv(B, H, Hkv, T, T, d, dtype, seed=T + w)
+    dout = inputs.upstream(B, H, T, d, dtype, seed=T + w)
+    scale = 1 / math.sqrt(d)
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    o = attn.prefill(qg, kg, vg, scale=scale, window=w, lse=lse)
+    got = attn.prefill_backward(qg, kg, vg, o, lse, dout.cuda(), scale=scale, window=w)
+    torch.cuda.synchronize()
+    ref = oracle.attention_backward(q, k, v, dout, scale=scale, window=w)
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        check(name, g.cpu(), r, dtype)
+
+
 def test_single_position():
     # one key: dq = dk = 0 and dv = the summed upstream rows (up to rounding)
     q, k, v = inputs.qkv(1, 4, 2, 1, 1, 64, BF16, seed=5)

@@ -235,6 +235,11 @@ def test_backward_rejects_unsupported_shapes(lib):
         assert backward(lib, ws=None, ws_bytes=0, **kwargs) == WORKSPACE
 
 
+def test_backward_local_rejects_a_negative_window(lib):
+    assert lib.attn_prefill_backward_local(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, BF16, 1,
+                                           4, 2, 300, 128, 0.125, -1, FAKE, 1 << 20, None) == INVALID
+
+
 def test_backward_workspace(lib):
     # two float32 row statistics per padded query row: 300 rows pad to 384
     need = lib.attn_prefill_backward_workspace_size(BF16, 2, 4, 2, 300, 128)

@@ -99,11 +99,12 @@ def prefill_backward_workspace_size(dtype, B, H, Hkv, T, d) -> int:
 
 
 def prefill_backward(q, k, v, out, lse, dout, *, scale: float, causal: bool = True, dq=None,
-                     dk=None, dv=None, workspace=None, stream=None):
+                     dk=None, dv=None, workspace=None, stream=None, window: int = 0):
     """Gradients of full-sequence attention.  q, out, dout [B,H,T,d]; k, v
     [B,Hkv,T,d]; lse float32 [B,H,T] as written by ``prefill`` for the same
-    inputs.  Returns (dq, dk, dv); dk and dv are summed over the query heads
-    that share each K/V head."""
+    inputs (and the same ``window``: w > 0 is local attention).  Returns
+    (dq, dk, dv); dk and dv are summed over the query heads that share each
+    K/V head."""
     torch = _torch()
     _check(q, k, v, out, lse, dout, dq, dk, dv, workspace)
     B, H, T, d = q.shape
@@ -121,6 +122,16 @@ def prefill_backward(q, k, v, out, lse, dout, *, scale: float, causal: bool = Tr
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if window:
+        if not causal:
+            raise ValueError("a local window is causal")
+        st = _lib.load().attn_prefill_backward_local(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+            _dtype_code(q), B, H, Hkv, T, d, float(scale), int(window), _ptr(workspace), ws_bytes,
+            _stream_handle(stream, q.device))
+        if st != _lib.OK:
+            raise AttnError(st, "attn_prefill_backward_local")
+        return dq, dk, dv
     st = _lib.load().attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                            _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                            _dtype_code(q), B, H, Hkv, T, d, float(scale),

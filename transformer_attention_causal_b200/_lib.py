@@ -24,7 +24,8 @@ KERNEL_NAMES = {KERNEL_NONE: "none", KERNEL_SIMT: "simt", KERNEL_TCGEN05: "tcgen
 
 EXPORTS = ("attn_prefill", "attn_cached", "attn_prefill_local", "attn_cached_local",
            "attn_cached_local_workspace_size", "attn_cached_paged", "attn_cached_paged_workspace_size",
-           "attn_prefill_backward", "attn_prefill_backward_workspace_size",
+           "attn_prefill_backward", "attn_prefill_backward_local",
+           "attn_prefill_backward_workspace_size",
            "attn_kv_append_rope", "attn_cached_workspace_size", "attn_prefill_plan",
            "attn_cached_plan", "attn_status_string", "attn_device_status",
            "attn_set_wait_timeout_ns", "attn_test_set_flags", "attn_version")
@@ -89,6 +90,10 @@ def load() -> ctypes.CDLL:
             lib.attn_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, c_int, i64, i64,
                                                   i64, i64, i64, f32, c_int, vp, ctypes.c_size_t,
                                                   vp]
+            lib.attn_prefill_backward_local.restype = c_int
+            lib.attn_prefill_backward_local.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, c_int, i64,
+                                                        i64, i64, i64, i64, f32, i64, vp,
+                                                        ctypes.c_size_t, vp]
             lib.attn_prefill_backward_workspace_size.restype = ctypes.c_size_t
             lib.attn_prefill_backward_workspace_size.argtypes = [c_int, i64, i64, i64, i64, i64]
             lib.attn_test_set_flags.restype = None

@@ -565,7 +565,7 @@ attn_status_t set_smem_once(K kern, size_t bytes, std::once_flag (&once)[8]) {
     return st;
 }
 
-template <typename T, int DCH>
+template <typename T, int DCH, bool WINDOW>
 attn_status_t launch_backward(const Problem& pb, BwdParams& bp, const void* q, const void* k,
                               const void* v, const void* dout, cudaStream_t stream) {
     if (get_encoder() != ATTN_OK) return ATTN_ERR_CUDA;
@@ -583,8 +583,8 @@ attn_status_t launch_backward(const Problem& pb, BwdParams& bp, const void* q, c
     static std::once_flag once_kv[8], once_q[8];
     constexpr size_t smem_kv = bwd_dkdv_smem_bytes<DCH>();
     constexpr size_t smem_q = bwd_dq_smem_bytes<DCH>();
-    auto kern_kv = bwd_dkdv_kernel<T, DCH>;
-    auto kern_q = bwd_dq_kernel<T, DCH>;
+    auto kern_kv = bwd_dkdv_kernel<T, DCH, WINDOW>;
+    auto kern_q = bwd_dq_kernel<T, DCH, WINDOW>;
     if (set_smem_once(kern_kv, smem_kv, once_kv) != ATTN_OK ||
         set_smem_once(kern_q, smem_q, once_q) != ATTN_OK)
         return ATTN_ERR_CUDA;
@@ -651,12 +651,16 @@ size_t attn_prefill_backward_workspace_size(attn_dtype_t dtype, int64_t B, int64
     return backward_ws_bytes(pb);
 }
 
-attn_status_t attn_prefill_backward(const void* q, const void* k, const void* v, const void* o,
-                                    const float* lse, const void* dout, void* dq, void* dk,
-                                    void* dv, attn_dtype_t dtype, int64_t B, int64_t H,
-                                    int64_t Hkv, int64_t T, int64_t d, float scale, int causal,
-                                    void* workspace, size_t workspace_bytes, void* stream) {
-    Problem pb{dtype, B, H, Hkv, T, T, T, d, 0, causal ? 1 : 0, false};
+}  // extern "C"
+
+namespace {
+
+attn_status_t prefill_backward(const void* q, const void* k, const void* v, const void* o,
+                               const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                               attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t T,
+                               int64_t d, float scale, int causal, int64_t window, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    Problem pb{dtype, B, H, Hkv, T, T, T, d, 0, causal ? 1 : 0, false, window};
     if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
     attn_status_t st = check_backward(pb);
     if (st != ATTN_OK) return st;
@@ -685,6 +689,8 @@ attn_status_t attn_prefill_backward(const void* q, const void* k, const void* v,
     bp.n_t = int((T + 127) / 128);
     bp.Tpad = bp.n_t * 128;
     bp.d = int(d); bp.causal = causal ? 1 : 0;
+    // a window covering every key is plain causal attention
+    bp.window = (window > 0 && window < T) ? int(window) : 0;
     bp.nl = static_cast<float*>(workspace);
     bp.dd = bp.nl + size_t(B * H) * bp.Tpad;
     bp.scale = scale;
@@ -696,11 +702,41 @@ attn_status_t attn_prefill_backward(const void* q, const void* k, const void* v,
         return bf16 ? launch_backward_simt<__nv_bfloat16>(bp, q, k, v, s)
                     : launch_backward_simt<__half>(bp, q, k, v, s);
     }
+    if (bp.window > 0) {
+        if (d <= 64)
+            return bf16 ? launch_backward<__nv_bfloat16, 1, true>(pb, bp, q, k, v, dout, s)
+                        : launch_backward<__half, 1, true>(pb, bp, q, k, v, dout, s);
+        return bf16 ? launch_backward<__nv_bfloat16, 2, true>(pb, bp, q, k, v, dout, s)
+                    : launch_backward<__half, 2, true>(pb, bp, q, k, v, dout, s);
+    }
     if (d <= 64)
-        return bf16 ? launch_backward<__nv_bfloat16, 1>(pb, bp, q, k, v, dout, s)
-                    : launch_backward<__half, 1>(pb, bp, q, k, v, dout, s);
-    return bf16 ? launch_backward<__nv_bfloat16, 2>(pb, bp, q, k, v, dout, s)
-                : launch_backward<__half, 2>(pb, bp, q, k, v, dout, s);
+        return bf16 ? launch_backward<__nv_bfloat16, 1, false>(pb, bp, q, k, v, dout, s)
+                    : launch_backward<__half, 1, false>(pb, bp, q, k, v, dout, s);
+    return bf16 ? launch_backward<__nv_bfloat16, 2, false>(pb, bp, q, k, v, dout, s)
+                : launch_backward<__half, 2, false>(pb, bp, q, k, v, dout, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_prefill_backward(const void* q, const void* k, const void* v, const void* o,
+                                    const float* lse, const void* dout, void* dq, void* dk,
+                                    void* dv, attn_dtype_t dtype, int64_t B, int64_t H,
+                                    int64_t Hkv, int64_t T, int64_t d, float scale, int causal,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    return prefill_backward(q, k, v, o, lse, dout, dq, dk, dv, dtype, B, H, Hkv, T, d, scale, causal, 0,
+                            workspace, workspace_bytes, stream);
+}
+
+attn_status_t attn_prefill_backward_local(const void* q, const void* k, const void* v, const void* o,
+                                          const float* lse, const void* dout, void* dq, void* dk,
+                                          void* dv, attn_dtype_t dtype, int64_t B, int64_t H,
+                                          int64_t Hkv, int64_t T, int64_t d, float scale,
+                                          int64_t window, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+    return prefill_backward(q, k, v, o, lse, dout, dq, dk, dv, dtype, B, H, Hkv, T, d, scale, 1, window,
+                            workspace, workspace_bytes, stream);
 }
 
 attn_status_t attn_cached(const void* q, const void* k_hist, const void* v_hist, void* o,

@@ -66,6 +66,7 @@ struct BwdParams {
     float* nl;            // workspace [B*H, Tpad]: -lse * log2(e); -inf on padding rows
     float* dd;            // workspace [B*H, Tpad]: D = sum_t dO*O; 0 on padding rows
     int B, H, Hkv, G, T, Tpad, d, causal;
+    int window;           // local window w (causal): row i reads keys i - w < j <= i; 0: none
     int n_t;              // ceil(T / 128)
     float scale, scale_log2;
     uint64_t timeout_ns;
@@ -200,7 +201,7 @@ __device__ __forceinline__ void bwd_store_row(uint32_t t_acc, int d, float mul, 
 
 // ------------------------------------------------------------------ dK, dV
 
-template <typename T, int DCH>
+template <typename T, int DCH, bool WINDOW>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -233,7 +234,9 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int kt = int(blockIdx.x / unsigned(p.B * p.Hkv));   // heaviest (kt = 0) first
     const int b = bk / p.Hkv, kvh = bk % p.Hkv;
     const int q_lo = p.causal ? kt : 0;
-    const int n_q = p.n_t - q_lo;
+    // with a window only the query tiles whose rows reach this key tile
+    const int q_hi = WINDOW ? min(p.n_t - 1, (kt * 128 + 127 + p.window - 1) / 128) : p.n_t - 1;
+    const int n_q = q_hi - q_lo + 1;
     const int n_it = p.G * n_q;
 
     if (threadIdx.x == 0) {
@@ -368,8 +371,11 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tmem_ld32(tS + 0, r[0]);
             tmem_ld32(tS + 32, r[1]);
             tmem_wait_ld();
-            // causal diagonal tile: query column i sees key row j only when i >= j
-            const int first_vis = ((p.causal && qt == kt) ? row : 0) - 64 * half;
+            // causal diagonal tile: query column i sees key row j only when i >= j;
+            // with a window also only while i - j < w
+            const int rel = row - (qt - kt) * 128 - 64 * half;   // column of i = j in this half
+            const int first_vis = (p.causal && qt == kt) ? rel : -64 * half - 1;
+            const int end_vis = WINDOW ? rel + p.window : 64;
             const float2 c2v = make_float2(c2, c2);
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
@@ -383,6 +389,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                           c2v, make_float2(nlv[2 * e], nlv[2 * e + 1]));
                     if (32 * ch + 2 * e < first_vis) x.x = -INFINITY;
                     if (32 * ch + 2 * e + 1 < first_vis) x.y = -INFINITY;
+                    if (WINDOW && 32 * ch + 2 * e >= end_vis) x.x = -INFINITY;
+                    if (WINDOW && 32 * ch + 2 * e + 1 >= end_vis) x.y = -INFINITY;
                     const float p0 = ex2(x.x), p1 = ex2(x.y);
                     r[ch][2 * e] = __float_as_uint(p0);
                     r[ch][2 * e + 1] = __float_as_uint(p1);
@@ -451,7 +459,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
 // ------------------------------------------------------------------ dQ
 
-template <typename T, int DCH>
+template <typename T, int DCH, bool WINDOW>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -489,7 +497,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int qt = p.n_t - 1 - int(blockIdx.x / unsigned(p.B * p.H));   // heaviest first
     const int b = bh / p.H, h = bh % p.H;
     const int bk = b * p.Hkv + h / p.G;
-    const int n_kv = p.causal ? qt + 1 : p.n_t;
+    // key tiles n_first .. n_first + n_kv - 1 (with a window: from the first
+    // key the tile's first row sees); loop counters run from 0
+    const int n_first = WINDOW ? max(0, qt * 128 - p.window + 1) / 128 : 0;
+    const int n_kv = (p.causal ? qt + 1 : p.n_t) - n_first;
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(q_full), 1);
@@ -551,7 +562,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     mbar_expect_tx(bar, TB);
                     const uint32_t dst = (which ? sV : sK) + st * TB;
                     for (int c = 0; c < DCH; ++c)
-                        tma_load_3d(dst + c * kChunkBytes, which ? &tmV : &tmK, bar, c * 64, m * 128, bk);
+                        tma_load_3d(dst + c * kChunkBytes, which ? &tmV : &tmK, bar, c * 64,
+                                    (n_first + m) * 128, bk);
                     ++issued[which];
                 }
             }
@@ -688,10 +700,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (lane == 0) mbar_arrive(smem_u32(s_read));
             // key j = 128 n + c is visible when j < T and (not causal or j <= i);
             // `last` is counted from this half's first column
+            const int nt = n_first + n;
             int last = 127;
-            if (n * 128 + 127 >= p.T) last = p.T - 1 - n * 128;
-            if (p.causal && n == qt) last = min(last, row);
+            if (nt * 128 + 127 >= p.T) last = p.T - 1 - nt * 128;
+            if (p.causal && nt == qt) last = min(last, row);
             last -= 64 * half;
+            // with a window keys at or below i - w are not seen either
+            const int first = WINDOW ? i - p.window + 1 - nt * 128 - 64 * half : -1;
             const float2 c2v = make_float2(c2, c2);
             const float2 nlv = make_float2(nl, nl);
 #pragma unroll
@@ -703,6 +718,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                           c2v, nlv);
                     if (32 * ch + 2 * e > last) x.x = -INFINITY;
                     if (32 * ch + 2 * e + 1 > last) x.y = -INFINITY;
+                    if (WINDOW && 32 * ch + 2 * e < first) x.x = -INFINITY;
+                    if (WINDOW && 32 * ch + 2 * e + 1 < first) x.y = -INFINITY;
                     r[ch][2 * e] = __float_as_uint(ex2(x.x));
                     r[ch][2 * e + 1] = __float_as_uint(ex2(x.y));
                 }

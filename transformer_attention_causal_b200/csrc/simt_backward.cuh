@@ -84,7 +84,8 @@ simt_bwd_dkdv_kernel(const BwdParams p, const SimtBwdPtrs in) {
         const T* gb = static_cast<const T*>(p.dout) + size_t(bh) * p.T * p.d;
         const float* nl = p.nl + size_t(bh) * p.Tpad;
         const float* dd = p.dd + size_t(bh) * p.Tpad;
-        for (int i = p.causal ? j : 0; i < p.T; ++i) {
+        const int i_end = p.window > 0 ? min(p.T, j + p.window) : p.T;
+        for (int i = p.causal ? j : 0; i < i_end; ++i) {
             float qr[kSimtBwdCols], gr[kSimtBwdCols];
             load_row<T>(qb + size_t(i) * p.d, p.d, lane, qr);
             load_row<T>(gb + size_t(i) * p.d, p.d, lane, gr);
@@ -123,7 +124,7 @@ simt_bwd_dq_kernel(const BwdParams p, const SimtBwdPtrs in) {
     const T* kb = static_cast<const T*>(in.k) + size_t(bk) * p.T * p.d;
     const T* vb = static_cast<const T*>(in.v) + size_t(bk) * p.T * p.d;
     const int j_end = p.causal ? i + 1 : p.T;
-    for (int j = 0; j < j_end; ++j) {
+    for (int j = p.window > 0 ? max(0, i - p.window + 1) : 0; j < j_end; ++j) {
         float kr[kSimtBwdCols], vr[kSimtBwdCols];
         load_row<T>(kb + size_t(j) * p.d, p.d, lane, kr);
         load_row<T>(vb + size_t(j) * p.d, p.d, lane, vr);
