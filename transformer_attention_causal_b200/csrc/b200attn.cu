@@ -13,6 +13,7 @@
 
 #include "b200attn.h"
 #include "decode_splitkv.cuh"
+#include "decode_mma.cuh"
 #include "kv_append.cuh"
 #include "prefill_backward.cuh"
 #include "prefill_tcgen05.cuh"
@@ -42,6 +43,7 @@ struct Problem {
     int causal;
     bool cached;  // attn_cached: split-KV decode allowed
     int64_t window = 0;  // local window (0: none); causal only
+    bool paged = false;  // attn_cached_paged: K/V in page pools
 };
 
 struct Plan {
@@ -49,6 +51,7 @@ struct Plan {
     // split-KV decode
     int R = 0, Rv = 0, nsplit = 1;
     bool wide = false;
+    bool mma = false;    // warp-level MMA decode kernel (contiguous cache)
     int64_t chunk = 0, kv_end = 0, k_lo = 0;
     size_t ws_bytes = 0;
     // tcgen05 prefill
@@ -92,8 +95,9 @@ void plan_decode(const Problem& pb, Plan& pl) {
     pl.R = next_pow2_at_least4(pl.Rv);
     // the wide kernel's three 120-key stages of K and V fit shared memory up to d = 128
     pl.wide = pl.R <= 8 && (pb.d == 64 || pb.d == 128);
-    const int stage_keys = pl.wide ? 120 : 64;
-    const int ctas_per_sm = pl.wide ? 1 : 2;
+    pl.mma = !pb.paged && (pb.d == 64 || pb.d == 128) && pl.Rv <= 16;
+    const int stage_keys = pl.mma ? kDecMmaTK : (pl.wide ? 120 : 64);
+    const int ctas_per_sm = pl.mma || pl.wide ? 1 : 2;
     pl.kv_end = std::min<int64_t>(pb.S, pb.start_pos + pb.Tq);
     // a local window: no row sees a key below the first row's window
     pl.k_lo = pb.window > 0 ? std::max<int64_t>(0, pb.start_pos - pb.window + 1) : 0;
@@ -323,6 +327,48 @@ attn_status_t launch_decode_D(int R, bool wide, const DecodeParams& dp, cudaStre
     }
 }
 
+template <typename T, int DCH, int NT, bool WINDOW>
+attn_status_t launch_decode_mma_k(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& dp,
+                                  cudaStream_t stream) {
+    constexpr size_t smem = DecMmaShape<DCH>::smem_bytes();
+    auto kern = decode_mma_kernel<T, DCH, NT, WINDOW>;
+    static std::once_flag once[8];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    attn_status_t st = ATTN_OK;
+    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
+    if (st != ATTN_OK) return st;
+    dim3 grid(unsigned(dp.nsplit), unsigned(dp.B * dp.Hkv));
+    kern<<<grid, kDecMmaThreads, smem, stream>>>(mk, mv, dp);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
+    if (dp.nsplit > 1) {
+        const int64_t rows = int64_t(dp.B) * dp.Hkv * dp.Rv;
+        decode_combine_kernel<T, 64 * DCH><<<unsigned((rows + 3) / 4), 128, 0, stream>>>(dp);
+        return launch_status();
+    }
+    return ATTN_OK;
+}
+
+template <typename T>
+attn_status_t launch_decode_mma(const Problem& pb, const DecodeParams& dp, cudaStream_t stream) {
+    if (get_encoder() != ATTN_OK) return ATTN_ERR_CUDA;
+    CUtensorMap mk, mv;
+    if (encode_rows(&mk, dp.k, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK ||
+        encode_rows(&mv, dp.v, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK)
+        return ATTN_ERR_CUDA;
+    const bool two = dp.Rv > 8, win = dp.window > 0;
+    if (pb.d == 64) {
+        if (two) return win ? launch_decode_mma_k<T, 1, 2, true>(mk, mv, dp, stream)
+                            : launch_decode_mma_k<T, 1, 2, false>(mk, mv, dp, stream);
+        return win ? launch_decode_mma_k<T, 1, 1, true>(mk, mv, dp, stream)
+                   : launch_decode_mma_k<T, 1, 1, false>(mk, mv, dp, stream);
+    }
+    if (two) return win ? launch_decode_mma_k<T, 2, 2, true>(mk, mv, dp, stream)
+                        : launch_decode_mma_k<T, 2, 2, false>(mk, mv, dp, stream);
+    return win ? launch_decode_mma_k<T, 2, 1, true>(mk, mv, dp, stream)
+               : launch_decode_mma_k<T, 2, 1, false>(mk, mv, dp, stream);
+}
+
 // A paged K/V cache: page pools, the page table and the per-sequence lengths.
 struct PagedKV {
     const int32_t* page_table = nullptr;
@@ -358,6 +404,7 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
         dp.max_pages = paged->max_pages;
         dp.num_pages = paged->num_pages;
     }
+    if (pl.mma && !paged) return launch_decode_mma<T>(pb, dp, stream);
     switch (pb.d) {
     case 64: return launch_decode_D<T, 64>(pl.R, pl.wide, dp, stream);
     case 128: return launch_decode_D<T, 128>(pl.R, pl.wide, dp, stream);
@@ -764,7 +811,7 @@ namespace {
 Problem paged_problem(attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t Tnew,
                       int64_t d, int64_t max_kv_len) {
     return Problem{dtype, B, H, Hkv, Tnew, max_kv_len, max_kv_len, d,
-                   max_kv_len - Tnew, 1, true};
+                   max_kv_len - Tnew, 1, true, 0, true};
 }
 
 }  // namespace
