@@ -95,7 +95,7 @@ void plan_decode(const Problem& pb, Plan& pl) {
     pl.R = next_pow2_at_least4(pl.Rv);
     // the wide kernel's three 120-key stages of K and V fit shared memory up to d = 128
     pl.wide = pl.R <= 8 && (pb.d == 64 || pb.d == 128);
-    pl.mma = !pb.paged && (pb.d == 64 || pb.d == 128) && pl.Rv <= 16;
+    pl.mma = (pb.d == 64 || pb.d == 128) && pl.Rv <= 16;
     const int stage_keys = pl.mma ? kDecMmaTK : (pl.wide ? 120 : 64);
     const int ctas_per_sm = pl.mma || pl.wide ? 1 : 2;
     pl.kv_end = std::min<int64_t>(pb.S, pb.start_pos + pb.Tq);
@@ -327,11 +327,11 @@ attn_status_t launch_decode_D(int R, bool wide, const DecodeParams& dp, cudaStre
     }
 }
 
-template <typename T, int DCH, int NT, bool WINDOW>
+template <typename T, int DCH, int NT, bool WINDOW, bool PAGED = false>
 attn_status_t launch_decode_mma_k(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& dp,
                                   cudaStream_t stream) {
     constexpr size_t smem = DecMmaShape<DCH>::smem_bytes();
-    auto kern = decode_mma_kernel<T, DCH, NT, WINDOW>;
+    auto kern = decode_mma_kernel<T, DCH, NT, WINDOW, PAGED>;
     static std::once_flag once[8];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -350,9 +350,22 @@ attn_status_t launch_decode_mma_k(const CUtensorMap& mk, const CUtensorMap& mv, 
 }
 
 template <typename T>
-attn_status_t launch_decode_mma(const Problem& pb, const DecodeParams& dp, cudaStream_t stream) {
+attn_status_t launch_decode_mma(const Problem& pb, const DecodeParams& dp, cudaStream_t stream,
+                                int64_t page_size = 0) {
     if (get_encoder() != ATTN_OK) return ATTN_ERR_CUDA;
     CUtensorMap mk, mv;
+    if (dp.paged) {
+        // the page pools as [num_pages * Hkv, P, d], boxes of min(P, 128) rows
+        const uint32_t rows = uint32_t(std::min<int64_t>(page_size, kDecMmaTK));
+        if (encode_rows(&mk, dp.k, pb.dt, pb.d, page_size, page_size, dp.num_pages * pb.Hkv, rows) != ATTN_OK ||
+            encode_rows(&mv, dp.v, pb.dt, pb.d, page_size, page_size, dp.num_pages * pb.Hkv, rows) != ATTN_OK)
+            return ATTN_ERR_CUDA;
+        if (pb.d == 64)
+            return dp.Rv > 8 ? launch_decode_mma_k<T, 1, 2, false, true>(mk, mv, dp, stream)
+                             : launch_decode_mma_k<T, 1, 1, false, true>(mk, mv, dp, stream);
+        return dp.Rv > 8 ? launch_decode_mma_k<T, 2, 2, false, true>(mk, mv, dp, stream)
+                         : launch_decode_mma_k<T, 2, 1, false, true>(mk, mv, dp, stream);
+    }
     if (encode_rows(&mk, dp.k, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK ||
         encode_rows(&mv, dp.v, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK)
         return ATTN_ERR_CUDA;
@@ -404,7 +417,7 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
         dp.max_pages = paged->max_pages;
         dp.num_pages = paged->num_pages;
     }
-    if (pl.mma && !paged) return launch_decode_mma<T>(pb, dp, stream);
+    if (pl.mma) return launch_decode_mma<T>(pb, dp, stream, paged ? (int64_t(1) << paged->page_shift) : 0);
     switch (pb.d) {
     case 64: return launch_decode_D<T, 64>(pl.R, pl.wide, dp, stream);
     case 128: return launch_decode_D<T, 128>(pl.R, pl.wide, dp, stream);

@@ -21,6 +21,12 @@
 // About four instructions per key.  K and V stages arrive by TMA with the
 // 128-byte swizzle (conflict-free ldmatrix rows); rows past the end of the
 // history are zero-filled by TMA and masked by position.
+// Paged variant: each 128-key stage is one TMA copy per page it spans (boxes
+// of min(P, 128) rows over the pools); rows past the sequence's end and
+// out-of-range page ids (reported) are read at an out-of-range coordinate and
+// come back zero-filled, and the rows of the sequence's last page past its
+// length, which a whole-page copy brings in, are zeroed in shared memory by
+// the warp that owns them before any MMA reads them.
 #pragma once
 
 #include "decode_splitkv.cuh"
@@ -44,7 +50,7 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t tile, int key, int d0) {
     return tile + uint32_t(d0 >> 6) * 16384u + uint32_t(key) * 128u + (uint32_t(u ^ (key & 7)) << 4);
 }
 
-template <typename T, int DCH, int NT, bool WINDOW>
+template <typename T, int DCH, int NT, bool WINDOW, bool PAGED>
 __global__ void __launch_bounds__(kDecMmaThreads, 1)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeParams p) {
@@ -66,8 +72,10 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     const int split = blockIdx.x;
     const int b = unit / p.Hkv;
     const int kvh = unit % p.Hkv;
+    int64_t start_pos = p.start_pos, kv_end = p.kv_end;
+    if constexpr (PAGED) decode_span(p, b, start_pos, kv_end);
     const int64_t k_begin = (WINDOW ? p.k_lo : 0) + int64_t(split) * p.chunk;
-    const int64_t k_end = min64(p.kv_end, k_begin + p.chunk);
+    const int64_t k_end = min64(kv_end, k_begin + p.chunk);
     const int nstages = k_end > k_begin ? int((k_end - k_begin + TK - 1) / TK) : 0;
 
     if (threadIdx.x == 0) {
@@ -95,9 +103,32 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                 mbar_expect_tx(full, 2 * TB);
                 const int32_t k0 = int32_t(k_begin + int64_t(it) * TK);
                 const uint32_t kt = base + uint32_t(st) * 2 * TB;
-                for (int c = 0; c < DCH; ++c) {
-                    tma_load_3d(kt + c * 16384u, &tmK, full, c * 64, k0, unit);
-                    tma_load_3d(kt + TB + c * 16384u, &tmV, full, c * 64, k0, unit);
+                if constexpr (PAGED) {
+                    const int rows = min(1 << p.page_shift, TK);
+                    for (int sub = 0; sub < TK / rows; ++sub) {
+                        const int64_t tok = int64_t(k0) + int64_t(sub) * rows;
+                        int64_t z = p.num_pages * p.Hkv;   // past the pools: zero fill
+                        int y = 0;
+                        if (tok < kv_end) {
+                            const int32_t phys = p.page_table[int64_t(b) * p.max_pages + (tok >> p.page_shift)];
+                            if (phys < 0 || phys >= p.num_pages) {
+                                atomicCAS(&g_device_status, 0u, kStatusBadIndex);
+                            } else {
+                                z = int64_t(phys) * p.Hkv + kvh;
+                                y = int(tok & ((int64_t(1) << p.page_shift) - 1));
+                            }
+                        }
+                        const uint32_t off = uint32_t(sub * rows) * 128u;
+                        for (int c = 0; c < DCH; ++c) {
+                            tma_load_3d(kt + c * 16384u + off, &tmK, full, c * 64, y, int32_t(z));
+                            tma_load_3d(kt + TB + c * 16384u + off, &tmV, full, c * 64, y, int32_t(z));
+                        }
+                    }
+                } else {
+                    for (int c = 0; c < DCH; ++c) {
+                        tma_load_3d(kt + c * 16384u, &tmK, full, c * 64, k0, unit);
+                        tma_load_3d(kt + TB + c * 16384u, &tmV, full, c * 64, k0, unit);
+                    }
                 }
                 issued = it + 1;
             }
@@ -134,7 +165,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         for (int rr = 0; rr < 2; ++rr) {
             const int r = nt * 8 + rsub + rr;
             rvalid[nt][rr] = r < p.Rv;
-            lim[nt][rr] = p.start_pos + (r % p.Tnew);
+            lim[nt][rr] = start_pos + (r % p.Tnew);
         }
     float m_run[NT][2], l_part[NT][2];
     float o[NT][NK][4];
@@ -154,6 +185,24 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         if (!mbar_wait(smem_u32(&bars[st]), (it / NST) & 1, p.timeout_ns, abort_flag)) break;
         const int64_t k0 = k_begin + int64_t(it) * TK;
         const uint32_t ks = base + uint32_t(st) * 2 * TB, vs = ks + TB;
+        if constexpr (PAGED) {
+            // V rows of this warp past the sequence's end: a whole-page copy may
+            // have brought in whatever the page holds there; their P is 0, so
+            // make them 0 too (0 * NaN would not be)
+            const int64_t first_bad = k_end - (k0 + kb);
+            if (first_bad < 16) {
+                for (int idx = lane; idx < 16 * DCH * 8; idx += 32) {
+                    const int key = idx / (DCH * 8);
+                    if (key < first_bad) continue;
+                    const int u = idx % (DCH * 8);
+                    const uint32_t a = vs + uint32_t(u >> 3) * 16384u + uint32_t(kb + key) * 128u + uint32_t(u & 7) * 16u;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+                }
+                // ordered before the TMA refill of this stage (async proxy)
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+        }
 
         // ---- S^T = K Q^T (fp32, 16 keys x RM rows)
         float s[NT][4];

@@ -118,6 +118,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
 }
 
+// Makes this thread's generic-proxy shared-memory writes ordered with later
+// async-proxy accesses (TMA copies, tensor-core operand reads) of the same
+// bytes once a barrier orders the two.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ warp-level MMA
 // (mma.sync: the right tool where a kernel is bound by HBM, not by the
 // tensor pipe; fragments as the PTX ISA defines them for m16n8k16.)
