@@ -76,8 +76,8 @@ WINDOW_WORKLOAD = "gqa_prefill_swa_bf16"
 PAGED_WORKLOAD = "gqa_decode_paged_bf16"
 BACKWARD_WORKLOAD = "gqa16x8_backward_bf16"
 TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
-KERNEL_SOURCES = {"tcgen05": "prefill_tcgen05.cuh", "splitkv": "decode_splitkv.cuh",
-                  "paged": "decode_splitkv.cuh",
+KERNEL_SOURCES = {"tcgen05": "prefill_tcgen05.cuh", "splitkv": "decode_mma.cuh",
+                  "paged": "decode_mma.cuh",
                   "simt": "simt_attn.cuh", "append": "kv_append.cuh",
                   "backward": "prefill_backward.cuh"}
 
