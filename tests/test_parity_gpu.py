@@ -151,6 +151,7 @@ CACHED_CASES = [
     (BF16, 2, 4, 4, 2, 1500, 1502, 1600, 256, "splitkv"),   # head size 256, two rows per K/V head
     (BF16, 1, 4, 1, 1, 19999, 20000, 20000, 128, "splitkv"),  # one long sequence: many splits
     (BF16, 2, 4, 2, 1, 0, 1, 1, 128, "splitkv"),            # first token
+    (F16, 2, 16, 1, 1, 1999, 2000, 2048, 64, "splitkv"),    # 16 rows per K/V head at d = 64
     (F16, 2, 8, 1, 200, 300, 500, 520, 128, "tcgen05"),     # MQA chunked prefill
     (BF16, 1, 4, 2, 64, 37, 101, 101, 80, "tcgen05"),       # unaligned start
     (BF16, 1, 2, 2, 100, 400, 600, 640, 64, "tcgen05"),     # history past the last query
