@@ -72,35 +72,10 @@ struct PrefillParams {
 constexpr int kPfThreads = 384;  // 12 warps
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 16-bit columns (one swizzle atom column)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
-// Of every 8 column pairs of an unmasked tile, this many take their
-// exponentials on the FMA pipe (exp2_fma2) instead of MUFU.
-constexpr int kEmuPairsPer8 = 3;
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
-}
-
-// 2^x for two values on the FMA/ALU pipes, relative error <= 1.1e-4 over
-// [-126, 16] (gen_exp2_poly.py): j = nearest integer via the 1.5*2^23
-// addition, f = x - j in [-1/2, 1/2], p(f) a degree-3 fit of 2^f with p(0) = 1,
-// and 2^j applied by adding j << 23 to the bits of p(f).  Inputs below -126
-// are clamped (their weights are < 2^-126 of the row's largest and vanish in
-// the fp32 sums); -inf must not reach this function.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-    constexpr float kC1 = 6.932829618e-01f, kC2 = 2.422109693e-01f, kC3 = 5.500890315e-02f;
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    x.x = fmaxf(x.x, -126.f);
-    x.y = fmaxf(x.y, -126.f);
-    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-    const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
-    const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
-    float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-    q = __ffma2_rn(q, f, make_float2(kC1, kC1));
-    q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
-    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 // Columns past `last` of a 32-column chunk of scores (fp32 bits) become -inf.
