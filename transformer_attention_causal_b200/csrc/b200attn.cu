@@ -28,9 +28,8 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<uint32_t> g_test_flags{0};
 
-// Planning constants for B200: 148 SMs.  The wide decode kernel runs one
-// 512-thread CTA per SM with 120-key stages; the compact one (large row
-// counts) two 160-thread CTAs per SM with 64-key stages.
+// Planning constant for B200: 148 SMs (the split plan fills the last wave of
+// CTAs; the device's own count is read at launch where it matters).
 constexpr int kPlanSMs = 148;
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -50,8 +49,7 @@ struct Plan {
     attn_kernel_t kernel = ATTN_KERNEL_NONE;
     // split-KV decode
     int R = 0, Rv = 0, nsplit = 1;
-    bool wide = false;
-    bool mma = false;    // warp-level MMA decode kernel (contiguous cache)
+    bool mma = false;    // warp-level MMA decode kernel (d = 64 or 128)
     int64_t chunk = 0, kv_end = 0, k_lo = 0;
     size_t ws_bytes = 0;
     // tcgen05 prefill
@@ -93,11 +91,11 @@ void plan_decode(const Problem& pb, Plan& pl) {
     const int64_t G = pb.H / pb.Hkv;
     pl.Rv = int(G * pb.Tq);
     pl.R = next_pow2_at_least4(pl.Rv);
-    // the wide kernel's three 120-key stages of K and V fit shared memory up to d = 128
-    pl.wide = pl.R <= 8 && (pb.d == 64 || pb.d == 128);
+    // d = 64 / 128: the MMA kernel (128-key stages, one CTA per SM); d = 256:
+    // the CUDA-core kernel (64-key stages, two CTAs per SM)
     pl.mma = (pb.d == 64 || pb.d == 128) && pl.Rv <= 16;
-    const int stage_keys = pl.mma ? kDecMmaTK : (pl.wide ? 120 : 64);
-    const int ctas_per_sm = pl.mma || pl.wide ? 1 : 2;
+    const int stage_keys = pl.mma ? kDecMmaTK : 64;
+    const int ctas_per_sm = pl.mma ? 1 : 2;
     pl.kv_end = std::min<int64_t>(pb.S, pb.start_pos + pb.Tq);
     // a local window: no row sees a key below the first row's window
     pl.k_lo = pb.window > 0 ? std::max<int64_t>(0, pb.start_pos - pb.window + 1) : 0;
@@ -271,27 +269,6 @@ attn_status_t launch_decode_RP(const DecodeParams& dp, cudaStream_t stream) {
     return ATTN_OK;
 }
 
-template <typename T, int D, int R, int MODE>
-attn_status_t launch_decode_wide_RP(const DecodeParams& dp, cudaStream_t stream) {
-    constexpr size_t smem = WideShape<D, R>::smem_bytes(sizeof(T));
-    auto kern = decode_wide_kernel<T, D, R, MODE>;
-    static std::once_flag once[8];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    attn_status_t st = ATTN_OK;
-    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
-    if (st != ATTN_OK) return st;
-    dim3 grid(unsigned(dp.nsplit), unsigned(dp.B * dp.Hkv));
-    kern<<<grid, 512, smem, stream>>>(dp);
-    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
-    if (dp.nsplit > 1) {
-        const int64_t rows = int64_t(dp.B) * dp.Hkv * dp.Rv;
-        decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, stream>>>(dp);
-        return launch_status();
-    }
-    return ATTN_OK;
-}
-
 template <typename T, int D, int R>
 attn_status_t launch_decode_R(const DecodeParams& dp, cudaStream_t stream) {
     if (dp.paged) return launch_decode_RP<T, D, R, kDecodePaged>(dp, stream);
@@ -299,30 +276,12 @@ attn_status_t launch_decode_R(const DecodeParams& dp, cudaStream_t stream) {
     return launch_decode_RP<T, D, R, kDecodePlain>(dp, stream);
 }
 
-template <typename T, int D, int R>
-attn_status_t launch_decode_wide_R(const DecodeParams& dp, cudaStream_t stream) {
-    if (dp.paged) return launch_decode_wide_RP<T, D, R, kDecodePaged>(dp, stream);
-    if (dp.window > 0) return launch_decode_wide_RP<T, D, R, kDecodeWindow>(dp, stream);
-    return launch_decode_wide_RP<T, D, R, kDecodePlain>(dp, stream);
-}
-
-template <typename T, int D>
-attn_status_t launch_decode_D(int R, bool wide, const DecodeParams& dp, cudaStream_t stream) {
-    if constexpr (D <= 128) {
-        if (wide) {
-            if (R == 4) return launch_decode_wide_R<T, D, 4>(dp, stream);
-            if (R == 8) return launch_decode_wide_R<T, D, 8>(dp, stream);
-            return ATTN_ERR_UNSUPPORTED;
-        }
-    } else {
-        if (wide) return ATTN_ERR_UNSUPPORTED;
-    }
+// The CUDA-core split-KV decode (d = 256; R = G * Tnew padded to 4 or 8).
+template <typename T>
+attn_status_t launch_decode_256(int R, const DecodeParams& dp, cudaStream_t stream) {
     switch (R) {
-    case 4: return launch_decode_R<T, D, 4>(dp, stream);
-    case 8: return launch_decode_R<T, D, 8>(dp, stream);
-    case 16:
-        if constexpr (D <= 128) return launch_decode_R<T, D, 16>(dp, stream);
-        return ATTN_ERR_UNSUPPORTED;
+    case 4: return launch_decode_R<T, 256, 4>(dp, stream);
+    case 8: return launch_decode_R<T, 256, 8>(dp, stream);
     default: return ATTN_ERR_UNSUPPORTED;
     }
 }
@@ -418,12 +377,8 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
         dp.num_pages = paged->num_pages;
     }
     if (pl.mma) return launch_decode_mma<T>(pb, dp, stream, paged ? (int64_t(1) << paged->page_shift) : 0);
-    switch (pb.d) {
-    case 64: return launch_decode_D<T, 64>(pl.R, pl.wide, dp, stream);
-    case 128: return launch_decode_D<T, 128>(pl.R, pl.wide, dp, stream);
-    case 256: return launch_decode_D<T, 256>(pl.R, pl.wide, dp, stream);
-    default: return ATTN_ERR_UNSUPPORTED;
-    }
+    if (pb.d == 256) return launch_decode_256<T>(pl.R, dp, stream);
+    return ATTN_ERR_UNSUPPORTED;
 }
 
 template <typename T, int DCH, bool WINDOW, bool PAGED = false>

@@ -1,5 +1,7 @@
-// Split-KV cached-decode attention: a few new query tokens per sequence
-// against a long K/V history.  HBM-bound: every call streams the visible
+// Split-KV cached-decode attention on CUDA cores: a few new query tokens per
+// sequence against a long K/V history.  Used for d = 256 (head sizes 64 and
+// 128 run on the warp-level MMA kernel of decode_mma.cuh, which shares this
+// file's parameters, span helper and combine kernel).  HBM-bound: every call streams the visible
 // history once ("Multi-query attention, annotated" §2.4.1: incremental
 // attention rereads the whole cache at about one multiply-add per number
 // read), so the kernel is built around keeping HBM busy, not around FLOPs.
@@ -562,372 +564,6 @@ decode_combine_kernel(const DecodeParams p) {
     }
     if (lane == 0 && p.lse)
         p.lse[orow] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
-}
-
-}  // namespace b200attn
-
-namespace b200attn {
-
-// ---------------------------------------------------------------------------
-// Wide split-KV decode: the same online-softmax split as
-// decode_splitkv_kernel, shaped for occupancy and instruction count.
-// 15 consumer warps + 1 producer warp per CTA (four warps on every SM
-// sub-partition, <= 128 registers each), 120-key stages (8 keys per consumer
-// warp).  Scores: a key row is split over LPK = D / EA lanes (EA elements =
-// one or two 16-byte pieces each, chosen so the pre-scaled queries take
-// R x EA = 64 registers), dot products in packed fp32x2 FMAs, one halving
-// shuffle reduction per group of 32 / LPK keys.  Weighted sum: all 32 lanes
-// split the head dimension (EC = D / 32 elements each) and walk the warp's
-// keys, so every lane holds only R x EC partial outputs.
-template <int D, int R>
-struct WideShape {
-    static constexpr int NW = 15;                      // consumer warps
-    static constexpr int KW = 8;                       // keys per warp per stage
-    static constexpr int TK = NW * KW;                 // keys per stage
-    static constexpr int NST = 3;                      // ring depth
-    static constexpr int EA0 = 64 / R;
-    static constexpr int EA = EA0 > D / 8 ? D / 8 : EA0;  // score elements per lane
-    static constexpr int LPK = D / EA;                 // lanes per key (scores)
-    static constexpr int KPG = 32 / LPK;               // keys per warp-wide group
-    static constexpr int GPW = KW / KPG;               // groups per warp per stage
-    static constexpr int EC = D / 32;                  // weighted-sum elements per lane
-    static constexpr int LPR = 32 / R;                 // lanes per row in the softmax step
-    static constexpr int SPL = KW / LPR;               // scores per lane in that step
-    static_assert(EA % 8 == 0 || EA == 4, "score pieces are 8 or 16 bytes");
-    static_assert(LPK >= 8 && LPK <= 32 && 32 % LPK == 0, "lanes per key");
-    static_assert(EC == 2 || EC == 4 || EC == 8, "weighted-sum piece");
-    static_assert(R <= LPK && KW % KPG == 0 && KW % LPR == 0 && SPL >= 1, "split");
-    static constexpr size_t smem_bytes(size_t esz) {
-        return 2 * NST * size_t(TK) * D * esz + size_t(NW) * KW * R * 4 + size_t(NW) * R * 4 +
-               (2 * NST + 2) * 8 + 64;
-    }
-};
-
-// n consecutive 16-bit elements (n = 2, 4, 8 or 16) widened to fp32.
-template <typename T, int N>
-__device__ __forceinline__ void load_elems(const T* src, float (&f)[N]) {
-    if constexpr (N == 16) {
-        const uint4 w0 = reinterpret_cast<const uint4*>(src)[0];
-        const uint4 w1 = reinterpret_cast<const uint4*>(src)[1];
-        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float2 v = unpack2<T>(w[i]);
-            f[2 * i] = v.x;
-            f[2 * i + 1] = v.y;
-        }
-    } else if constexpr (N == 8) {
-        const uint4 w0 = *reinterpret_cast<const uint4*>(src);
-        const uint32_t w[4] = {w0.x, w0.y, w0.z, w0.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 v = unpack2<T>(w[i]);
-            f[2 * i] = v.x;
-            f[2 * i + 1] = v.y;
-        }
-    } else if constexpr (N == 4) {
-        const uint2 w0 = *reinterpret_cast<const uint2*>(src);
-        const float2 a = unpack2<T>(w0.x), b = unpack2<T>(w0.y);
-        f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-    } else {
-        const float2 a = unpack2<T>(*reinterpret_cast<const uint32_t*>(src));
-        f[0] = a.x; f[1] = a.y;
-    }
-}
-
-template <typename T, int D, int R, int MODE>
-__global__ void __launch_bounds__(512, 1)
-decode_wide_kernel(const DecodeParams p) {
-    constexpr bool PAGED = MODE == kDecodePaged;
-    constexpr bool WINDOW = MODE == kDecodeWindow;
-    using Sh = WideShape<D, R>;
-    constexpr int NW = Sh::NW, TK = Sh::TK, NST = Sh::NST, KW = Sh::KW, EA = Sh::EA, LPK = Sh::LPK,
-                  KPG = Sh::KPG, GPW = Sh::GPW, EC = Sh::EC, LPR = Sh::LPR, SPL = Sh::SPL;
-    extern __shared__ __align__(128) unsigned char smem[];
-    T* ks = reinterpret_cast<T*>(smem);                              // [NST][TK][D]
-    T* vs = ks + size_t(NST) * TK * D;                               // [NST][TK][D]
-    float* sc = reinterpret_cast<float*>(vs + size_t(NST) * TK * D); // [NW][KW][R]
-    float* al = sc + NW * KW * R;                                    // [NW][R]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(al + NW * R);       // full[NST], empty[NST]
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * NST);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int unit = blockIdx.y;
-    const int split = blockIdx.x;
-    const int b = unit / p.Hkv;
-    const int kvh = unit % p.Hkv;
-    int64_t start_pos = p.start_pos, kv_end = p.kv_end;
-    if constexpr (PAGED) decode_span(p, b, start_pos, kv_end);
-    const int64_t k_begin = (WINDOW ? p.k_lo : 0) + int64_t(split) * p.chunk;
-    const int64_t k_end = min64(kv_end, k_begin + p.chunk);
-    const int nstages = k_end > k_begin ? int((k_end - k_begin + TK - 1) / TK) : 0;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(smem_u32(&bars[s]), 1);
-            mbar_init(smem_u32(&bars[NST + s]), NW);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    const T* kg = static_cast<const T*>(p.k) + (size_t(unit) * p.S_cap) * D;
-    const T* vg = static_cast<const T*>(p.v) + (size_t(unit) * p.S_cap) * D;
-
-    if (warp == NW) {
-        if constexpr (!PAGED) {
-            if (lane == 0) producer_contiguous<T, D, TK, NST>(p, nstages, k_begin, k_end, kg, vg, ks, vs,
-                                                              bars, abort_flag);
-            return;
-        }
-        int issued = 0;
-        const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : nstages;
-        for (int it = 0; it < n_loads; ++it) {
-            const int st = it % NST;
-            bool ok = true;
-            if (lane == 0)
-                ok = mbar_wait(smem_u32(&bars[NST + st]), ((it / NST) & 1) ^ 1, p.timeout_ns, abort_flag);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            issued = it + 1;
-            const int64_t k0 = k_begin + int64_t(it) * TK;
-            const int n = int(min64(TK, k_end - k0));
-            const uint32_t full = smem_u32(&bars[st]);
-            if (lane == 0) mbar_expect_tx(full, 2 * uint32_t(n) * D * sizeof(T));
-            load_kv_rows<T, D>(p, lane, b, kvh, kg, vg, k0, n, ks + size_t(st) * TK * D,
-                               vs + size_t(st) * TK * D, full);
-        }
-        if (lane == 0)
-            for (int it = issued - 1; it >= 0 && it >= issued - NST; --it)
-                mbar_wait(smem_u32(&bars[it % NST]), (it / NST) & 1, p.timeout_ns, nullptr);
-        return;
-    }
-
-    const int sub = lane % LPK;
-    const int kslot = lane / LPK;
-    const int my_row = sub / (LPK / R);
-    // score pieces: EA elements per lane, split into 16-byte pieces spread
-    // LPK * 8 elements apart (conflict-free quarter-warp reads)
-    constexpr int NPC = EA >= 8 ? EA / 8 : 1;          // pieces per lane
-    constexpr int PE = EA >= 8 ? 8 : EA;               // elements per piece
-
-    float2 q2[R][EA / 2];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const bool valid = r < p.Rv;
-        const int g = valid ? r / p.Tnew : 0;
-        const int t = valid ? r % p.Tnew : 0;
-        const T* qrow = static_cast<const T*>(p.q) +
-                        ((size_t(b) * p.H + size_t(kvh) * p.G + g) * p.Tnew + t) * D;
-#pragma unroll
-        for (int c = 0; c < NPC; ++c) {
-            float f[PE];
-            load_elems<T, PE>(qrow + (c * LPK + sub) * PE, f);
-#pragma unroll
-            for (int j = 0; j < PE / 2; ++j)
-                q2[r][c * (PE / 2) + j] =
-                    valid ? make_float2(f[2 * j] * p.scale_log2, f[2 * j + 1] * p.scale_log2)
-                          : make_float2(0.f, 0.f);
-        }
-    }
-    // one new token: every key in [k_lo, kv_end) is visible (window included)
-    const bool single = p.Tnew == 1;
-    int64_t row_lim[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) row_lim[r] = (r < p.Rv) ? start_pos + (r % p.Tnew) : -1;
-
-    float2 o2[R][EC / 2];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int j = 0; j < EC / 2; ++j) o2[r][j] = make_float2(0.f, 0.f);
-    const int rb = lane / LPR;
-    float m_run = -INFINITY, l_part = 0.f;
-    float* scw = sc + warp * KW * R;
-    float* alw = al + warp * R;
-
-    for (int it = 0; it < nstages; ++it) {
-        const int st = it % NST;
-        if (!mbar_wait(smem_u32(&bars[st]), (it / NST) & 1, p.timeout_ns, abort_flag)) break;
-        const int64_t k0 = k_begin + int64_t(it) * TK;
-        const int nvalid = int(min64(TK, k_end - k0));
-        const T* kst = ks + size_t(st) * TK * D;
-        const T* vst = vs + size_t(st) * TK * D;
-
-        // A. scores
-#pragma unroll
-        for (int gi = 0; gi < GPW; ++gi) {
-            const int kw = gi * KPG + kslot;
-            const int ki = warp * KW + kw;
-            float acc[R];
-            float2 a2[R];
-#pragma unroll
-            for (int c = 0; c < NPC; ++c) {
-                float f[PE];
-                load_elems<T, PE>(kst + size_t(ki) * D + (c * LPK + sub) * PE, f);
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-#pragma unroll
-                    for (int j = 0; j < PE / 2; ++j) {
-                        const float2 kv = make_float2(f[2 * j], f[2 * j + 1]);
-                        if (c == 0 && j == 0) a2[r] = __fmul2_rn(q2[r][0], kv);
-                        else a2[r] = __ffma2_rn(q2[r][c * (PE / 2) + j], kv, a2[r]);
-                    }
-            }
-#pragma unroll
-            for (int r = 0; r < R; ++r) acc[r] = a2[r].x + a2[r].y;
-            int n = R;
-#pragma unroll
-            for (int o = LPK / 2; o >= 1; o >>= 1) {
-                if (n > 1) {
-                    const bool upper = (lane & o) != 0;
-#pragma unroll
-                    for (int i = 0; i < R / 2; ++i) {
-                        if (i < n / 2) {
-                            const float send = upper ? acc[i] : acc[i + n / 2];
-                            const float keep = upper ? acc[i + n / 2] : acc[i];
-                            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-                        }
-                    }
-                    n >>= 1;
-                } else {
-                    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
-                }
-            }
-            bool vis = ki < nvalid;
-            if (!single) {
-                const int64_t wnd = WINDOW ? p.window : (int64_t(1) << 62);
-                const int64_t j = k0 + ki;
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-                    if (r == my_row) vis = vis && (j <= row_lim[r]) && (!WINDOW || j > row_lim[r] - wnd);
-            }
-            if (sub % (LPK / R) == 0) scw[kw * R + my_row] = vis ? acc[0] : -INFINITY;
-        }
-        __syncwarp();
-
-        // B. online softmax over the warp's KW keys, row rb
-        {
-            float s[SPL];
-            float mx = -INFINITY;
-#pragma unroll
-            for (int e = 0; e < SPL; ++e) {
-                s[e] = scw[((lane % LPR) * SPL + e) * R + rb];
-                mx = fmaxf(mx, s[e]);
-            }
-#pragma unroll
-            for (int o = LPR / 2; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            const float m_new = fmaxf(m_run, mx);
-            float alpha = 1.f, psum = 0.f;
-            if (m_new != -INFINITY) {
-                alpha = ex2(m_run - m_new);
-#pragma unroll
-                for (int e = 0; e < SPL; ++e) {
-                    s[e] = ex2(s[e] - m_new);
-                    psum += s[e];
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < SPL; ++e) s[e] = 0.f;
-            }
-            l_part = l_part * alpha + psum;
-            m_run = m_new;
-#pragma unroll
-            for (int e = 0; e < SPL; ++e) scw[((lane % LPR) * SPL + e) * R + rb] = s[e];
-            if (lane % LPR == 0) alw[rb] = alpha;
-        }
-        __syncwarp();
-
-        // C. rescale and accumulate P V: lanes split d, each walks the warp's keys
-        {
-            float a[R];
-            bool any = false;
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                a[r] = alw[r];
-                any |= (a[r] != 1.f);
-            }
-            if (any) {
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-#pragma unroll
-                    for (int jj = 0; jj < EC / 2; ++jj) o2[r][jj] = __fmul2_rn(o2[r][jj], make_float2(a[r], a[r]));
-            }
-            const int kv_here = min(KW, nvalid - warp * KW);
-#pragma unroll
-            for (int kw = 0; kw < KW; ++kw) {
-                if (kw < kv_here) {
-                    float pr[R];
-#pragma unroll
-                    for (int r = 0; r < R; ++r) pr[r] = scw[kw * R + r];
-                    float f[EC];
-                    load_elems<T, EC>(vst + size_t(warp * KW + kw) * D + lane * EC, f);
-#pragma unroll
-                    for (int r = 0; r < R; ++r)
-#pragma unroll
-                        for (int jj = 0; jj < EC / 2; ++jj)
-                            o2[r][jj] = __ffma2_rn(make_float2(pr[r], pr[r]),
-                                                   make_float2(f[2 * jj], f[2 * jj + 1]), o2[r][jj]);
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars[NST + st]));
-    }
-
-    // ---- merge the warps of the CTA
-#pragma unroll
-    for (int o = LPR / 2; o >= 1; o >>= 1) l_part += __shfl_xor_sync(0xffffffffu, l_part, o);
-
-    asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
-    float* mo = reinterpret_cast<float*>(smem);  // [NW][R]
-    float* lo = mo + NW * R;                     // [NW][R]
-    float* oo = lo + NW * R;                     // [NW][R][D]
-    if (lane % LPR == 0) {
-        mo[warp * R + rb] = m_run;
-        lo[warp * R + rb] = l_part;
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int jj = 0; jj < EC / 2; ++jj) {
-            oo[(warp * R + r) * D + lane * EC + 2 * jj] = o2[r][jj].x;
-            oo[(warp * R + r) * D + lane * EC + 2 * jj + 1] = o2[r][jj].y;
-        }
-    asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
-
-    const bool aborted = *abort_flag != 0;
-    for (int idx = threadIdx.x; idx < p.Rv * D; idx += NW * 32) {
-        const int r = idx / D, e = idx % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, mo[w * R + r]);
-        float L = 0.f, acc = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float f = ex2(mo[w * R + r] - M);
-                L += f * lo[w * R + r];
-                acc += f * oo[(w * R + r) * D + e];
-            }
-        }
-        if (aborted) continue;
-        if (p.nsplit == 1) {
-            const int g = r / p.Tnew, t = r % p.Tnew;
-            const size_t orow = (size_t(b) * p.H + size_t(kvh) * p.G + g) * p.Tnew + t;
-            static_cast<T*>(p.o)[orow * D + e] = from_f32<T>(L > 0.f ? acc / L : 0.f);
-            if (e == 0 && p.lse)
-                p.lse[orow] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
-        } else {
-            const size_t pi = (size_t(unit) * p.nsplit + split) * p.Rv + r;
-            p.ws_o[pi * D + e] = acc;
-            if (e == 0) {
-                p.ws_m[pi] = M;
-                p.ws_l[pi] = L;
-            }
-        }
-    }
 }
 
 }  // namespace b200attn
