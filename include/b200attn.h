@@ -316,8 +316,9 @@ ATTN_API attn_status_t attn_device_status(void* stream, int reset);
 ATTN_API void attn_set_wait_timeout_ns(uint64_t ns);
 
 /* Test hook for the device timeout path (no counterpart in the pages):
- * flags & 1 makes the K/V producers of the tensor-core and split-KV kernels
- * issue no copies, so every bounded wait on them runs out, the kernel
+ * flags & 1 makes the TMA producers of the tensor-core prefill, backward and
+ * split-KV decode kernels issue no copies, so every bounded wait on them runs
+ * out, the kernel
  * records ATTN_ERR_DEVICE_TIMEOUT and exits cleanly (its output is then
  * undefined).  0 restores normal operation.  Read at launch; not for
  * production use. */

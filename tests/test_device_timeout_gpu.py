@@ -1,6 +1,6 @@
 """Device-side failure detection without a GPU fault (needs a B200).
 
-Every wait inside the kernels is bounded.  The test hook makes the K/V
+Every wait inside the kernels is bounded.  The test hook makes the TMA
 producers issue no copies, so the consumers' waits run out after a short
 limit: the kernels must record ATTN_ERR_DEVICE_TIMEOUT, exit cleanly (TMEM
 freed, no copy left in flight) and leave the context usable, which the normal
@@ -15,6 +15,7 @@ import torch
 
 import transformer_attention_causal_b200 as attn
 from oracle import attention as oracle
+from oracle import attention_backward as oracle_backward
 from transformer_attention_causal_b200 import _lib, inputs
 
 pytestmark = pytest.mark.gpu
@@ -57,4 +58,33 @@ def test_bounded_waits_report_a_timeout_and_leave_the_context_usable():
     ref = oracle(dq.cpu(), dk.cpu(), dv.cpu(), scale=scale, causal=True, start_pos=999)
     err = np.abs(out - ref)
     assert err.max() <= 1.5e-2 and err.mean() <= 2e-3
+    assert attn.device_status() == _lib.OK
+
+
+@pytest.mark.parametrize("window", [0, 100])
+def test_backward_waits_report_a_timeout_and_leave_the_context_usable(window):
+    """Both backward kernels (dK/dV and dQ) under the no-copy hook."""
+    lib = _lib.load()
+    scale = 1 / math.sqrt(128)
+    B, H, Hkv, T, d = 1, 4, 2, 300, 128
+    q, k, v = inputs.qkv(B, H, Hkv, T, T, d, torch.bfloat16, seed=33)
+    dout = inputs.upstream(B, H, T, d, torch.bfloat16, seed=33)
+    qg, kg, vg, dog = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    o = attn.prefill(qg, kg, vg, scale=scale, lse=lse, window=window)
+    assert attn.device_status(reset=True) == _lib.OK
+    try:
+        attn.set_wait_timeout_ns(20_000_000)  # 20 ms
+        lib.attn_test_set_flags(1)
+        attn.prefill_backward(qg, kg, vg, o, lse, dog, scale=scale, window=window)
+        assert attn.device_status(reset=True) == _lib.ERR_DEVICE_TIMEOUT
+    finally:
+        lib.attn_test_set_flags(0)
+        attn.set_wait_timeout_ns(0)
+    grads = attn.prefill_backward(qg, kg, vg, o, lse, dog, scale=scale, window=window)
+    torch.cuda.synchronize()
+    ref = oracle_backward(q, k, v, dout, scale=scale, causal=True, window=window)
+    for g, r in zip(grads, ref):
+        g = g.double().cpu().numpy()
+        assert np.linalg.norm(g - r) <= 2 * 2.0 ** -8 * np.linalg.norm(r)
     assert attn.device_status() == _lib.OK

@@ -711,6 +711,7 @@ attn_status_t prefill_backward(const void* q, const void* k, const void* v, cons
     bp.scale = scale;
     bp.scale_log2 = scale * 1.4426950408889634f;
     bp.timeout_ns = g_timeout_ns.load();
+    bp.test_flags = g_test_flags.load();
     const bool bf16 = dtype == ATTN_BF16;
     if (!backward_on_tensor_cores(pb)) {
         if (dtype == ATTN_F32) return launch_backward_simt<float>(bp, q, k, v, s);

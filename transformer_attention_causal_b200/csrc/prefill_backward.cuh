@@ -70,6 +70,7 @@ struct BwdParams {
     int n_t;              // ceil(T / 128)
     float scale, scale_log2;
     uint64_t timeout_ns;
+    uint32_t test_flags;  // kTestSkipLoads: issue no copies (timeout-path tests)
 };
 
 constexpr int kBwdThreads = 384;  // 12 warps: producer, MMA, 2 idle, 8 elementwise
@@ -265,9 +266,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (warp == 0) {
         // ================================================= TMA producer
         if (lane == 0) {
+            const bool skip = p.test_flags & kTestSkipLoads;
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmdO);
-            {
+            if (!skip) {
                 const uint32_t bar = smem_u32(kv_full);
                 mbar_expect_tx(bar, 2 * TB);
                 for (int c = 0; c < DCH; ++c) {
@@ -276,7 +278,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
             }
             int it = 0;
-            for (; it < n_it; ++it) {
+            for (; it < n_it && !skip; ++it) {
                 const int st = it % NQ;
                 if (!mbar_wait(smem_u32(&q_empty[st]), ((it / NQ) & 1) ^ 1, p.timeout_ns, abort_flag)) break;
                 const int h = kvh * p.G + it / n_q;
@@ -293,7 +295,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 bulk_load(smem_u32(rowstat + st * 256 + 128), p.dd + ro, 512, bar);
             }
             // no copy may still be landing when the CTA exits
-            mbar_wait(smem_u32(kv_full), 0, p.timeout_ns, nullptr);
+            if (!skip) mbar_wait(smem_u32(kv_full), 0, p.timeout_ns, nullptr);
             for (int i = it - 1; i >= 0 && i >= it - NQ; --i)
                 mbar_wait(smem_u32(&q_full[i % NQ]), (i / NQ) & 1, p.timeout_ns, nullptr);
         }
@@ -535,9 +537,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (warp == 0) {
         // ================================================= TMA producer
         if (lane == 0) {
+            const bool skip = p.test_flags & kTestSkipLoads;
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            {
+            if (!skip) {
                 const uint32_t bar = smem_u32(q_full);
                 mbar_expect_tx(bar, 2 * TB);
                 for (int c = 0; c < DCH; ++c) {
@@ -547,7 +550,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             // K_m and V_m into their own rings, in tile order
             int issued[2] = {0, 0};   // K and V copies issued
-            bool kv_ok = true;
+            bool kv_ok = !skip;
             for (int m = 0; m < n_kv && kv_ok; ++m) {
                 for (int which = 0; which < 2 && kv_ok; ++which) {
                     const int nst = which ? NVR : NKR;
@@ -568,7 +571,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
             }
             // no copy may still be landing when the CTA exits
-            mbar_wait(smem_u32(q_full), 0, p.timeout_ns, nullptr);
+            if (!skip) mbar_wait(smem_u32(q_full), 0, p.timeout_ns, nullptr);
             for (int i = issued[0] - 1; i >= 0 && i >= issued[0] - NKR; --i)
                 mbar_wait(smem_u32(&k_full[i % NKR]), (i / NKR) & 1, p.timeout_ns, nullptr);
             for (int i = issued[1] - 1; i >= 0 && i >= issued[1] - NVR; --i)
