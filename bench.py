@@ -798,7 +798,7 @@ def run_reference(args, dist_ctx):
     value = tot_w / tot_s
     unit = sample.unit
     line = {
-        "metric": METRIC, "impl": "reference", "value": value, "unit": unit, "n_gpus": 0,
+        "metric": METRIC, "impl": "reference", "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
