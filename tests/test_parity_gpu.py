@@ -238,6 +238,28 @@ def test_rows_with_large_logits():
     assert_close(f64(got).reshape(B * H, -1), ref.reshape(B * H, -1), BF16)
 
 
+@pytest.mark.parametrize("case", [
+    # B, H, Hkv, Tnew, start_pos, S, kernel
+    (2, 8, 2, 1, 1499, 1500, "splitkv"),     # decode: the MMA kernel's lazy rescale
+    (1, 4, 1, 4, 996, 1000, "splitkv"),      # several new rows per K/V head
+    (1, 4, 2, 200, 500, 700, "tcgen05"),     # chunked prefill
+], ids=lambda c: "-".join(map(str, c)))
+def test_cached_rows_with_large_logits(case):
+    """Cached attention with the scores scaled up 50x and keys growing along
+    the sequence, so the running maximum keeps rising from split to split and
+    tile to tile."""
+    B, H, Hkv, Tnew, st, S, kernel = case
+    d = 128
+    assert attn.cached_plan(BF16, B, H, Hkv, Tnew, S, S, d, st) == kernel
+    q, k, v = inputs.qkv(B, H, Hkv, Tnew, S, d, BF16, seed=13)
+    ramp = torch.linspace(0.5, 4.0, S).reshape(1, 1, S, 1)
+    k = (k.float() * ramp).to(BF16)
+    scale = 50.0 / math.sqrt(d)
+    got = gpu_cached(q, k, v, st, scale)
+    ref = oracle(q, k, v, scale=scale, causal=True, start_pos=st)
+    assert_close(f64(got).reshape(B * H, -1), ref.reshape(B * H, -1), BF16)
+
+
 def test_empty_problem_leaves_output_untouched():
     q = torch.zeros((0, 4, 8, 64), dtype=BF16, device="cuda")
     out = attn.prefill(q, q.new_zeros((0, 2, 8, 64)), q.new_zeros((0, 2, 8, 64)), scale=0.1)

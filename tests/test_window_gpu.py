@@ -121,3 +121,26 @@ def test_full_size_windowed_prefill_sampled_rows():
     ref = oracle.attention(q, k, v, scale=1 / math.sqrt(d), causal=True, window=w, rows=rows)
     flat = got.reshape(B * H * T, d)[torch.as_tensor(rows)]
     check(flat.reshape(1, len(rows), d), ref.reshape(1, len(rows), d), BF16)
+
+
+@pytest.mark.parametrize("kind", ["prefill", "decode"])
+def test_window_with_large_logits(kind):
+    """Scores scaled up 50x with keys growing along the sequence: within a
+    window the running maximum keeps rising, and the keys that leave the
+    window are the small ones."""
+    d, w = 128, 300
+    if kind == "prefill":
+        B, H, Hkv, T, S, st = 1, 4, 2, 900, 900, 0
+    else:
+        B, H, Hkv, T, S, st = 2, 8, 2, 1, 2000, 1999
+    q, k, v = inputs.qkv(B, H, Hkv, T, S, d, BF16, seed=21)
+    ramp = torch.linspace(0.5, 4.0, S).reshape(1, 1, S, 1)
+    k = (k.float() * ramp).to(BF16)
+    scale = 50.0 / math.sqrt(d)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    if kind == "prefill":
+        got = attn.prefill(qd, kd, vd, scale=scale, window=w)
+    else:
+        got = attn.cached(qd, kd, vd, start_pos=st, scale=scale, window=w)
+    ref = oracle.attention(q, k, v, scale=scale, causal=True, start_pos=st, window=w)
+    check(got, ref, BF16)

@@ -388,11 +388,19 @@ attn_status_t launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk
     constexpr size_t smem = prefill_smem_bytes<DCH>();
     auto kern = prefill_tcgen05_kernel<T, DCH, WINDOW, PAGED>;
     static std::once_flag once[8];
+    static attn_status_t ready[8];
     int dev = 0;
     cudaGetDevice(&dev);
-    attn_status_t st = ATTN_OK;
-    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
-    if (st != ATTN_OK) return st;
+    std::call_once(once[dev & 7], [&] {
+        attn_status_t r = set_smem(kern, smem);
+        // the kernel's register split must fit the block's launch allocation,
+        // or its increase would never be granted
+        cudaFuncAttributes fa{};
+        if (r == ATTN_OK && cudaFuncGetAttributes(&fa, kern) != cudaSuccess) r = ATTN_ERR_CUDA;
+        if (r == ATTN_OK && fa.numRegs * kPfThreads < 128 * kPfRegsLow + 256 * kPfRegsHigh) r = ATTN_ERR_CUDA;
+        ready[dev & 7] = r;
+    });
+    if (ready[dev & 7] != ATTN_OK) return ready[dev & 7];
     kern<<<unsigned(grid), kPfThreads, smem, stream>>>(mq, mk, mv, pp);
     return launch_status();
 }

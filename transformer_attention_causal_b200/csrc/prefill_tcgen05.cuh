@@ -70,6 +70,10 @@ struct PrefillParams {
 };
 
 constexpr int kPfThreads = 384;  // 12 warps
+// Register split: warpgroup 0 (producer, issuer, two idle warps) gives
+// registers up, the two softmax warpgroups (a row of 128 scores per thread)
+// take them.  Needs launch registers x 384 >= 128 x low + 256 x high.
+constexpr int kPfRegsLow = 120, kPfRegsHigh = 192;
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 16-bit columns (one swizzle atom column)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -345,170 +349,173 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-
-    if (warp == 0) {
-        // ================================================= TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            uint32_t qcount[2] = {0, 0};   // Q loads per slot so far
-            int64_t li = 0;                // K/V loads so far (ring position)
-            bool ok = true;
-            for (int pass = 0; ok; ++pass) {
-                const int unit = prefill_pass_unit(pass);
-                if (unit >= n_units) break;
-                int b, kvh;
-                SlotInfo slot[2];
-                prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
-                const int nmax = max(slot[0].n_kv, slot[1].n_kv);
-                const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
-                                 : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    if (slot[s].n_kv == 0) continue;
-                    // the previous unit's Q.K^T MMAs of this slot are done with Q
-                    if (qcount[s] > 0 &&
-                        !mbar_wait(smem_u32(&q_empty[s]), (qcount[s] - 1) & 1, p.timeout_ns, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t bar = smem_u32(&q_full[s]);
-                    mbar_expect_tx(bar, DCH * kChunkBytes);
-                    for (int c = 0; c < DCH; ++c)
-                        tma_load_3d(sQ + (s * DCH + c) * kChunkBytes, &tmQ, bar, c * 64, slot[s].q0,
-                                    b * p.H + slot[s].h);
-                    ++qcount[s];
-                }
-                const int zkv = b * p.Hkv + kvh;
-                const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * (nmax - nmin);
-                for (int i = 0; i < n_loads && ok; ++i, ++li) {
-                    const int st = int(li % NST);
-                    if (!mbar_wait(smem_u32(&kv_empty[st]), uint32_t((li / NST) & 1) ^ 1, p.timeout_ns,
-                                   abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t bar = smem_u32(&kv_full[st]);
-                    mbar_expect_tx(bar, DCH * kChunkBytes);
-                    const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
-                    if (PAGED)
-                        load_kv_paged<DCH>(p, sRing + st * DCH * kChunkBytes, map, bar, nmin + (i >> 1), b,
-                                           kvh, slot[0].S);
-                    else
-                        for (int c = 0; c < DCH; ++c)
-                            tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64,
-                                        (nmin + (i >> 1)) * 128, zkv);
-                }
-            }
-            // no copy may still be landing in shared memory when the CTA exits
-            for (int64_t i = li - 1; i >= 0 && i >= li - NST; --i)
-                mbar_wait(smem_u32(&kv_full[i % NST]), uint32_t((i / NST) & 1), p.timeout_ns, nullptr);
-            for (int s = 0; s < 2; ++s)
-                if (qcount[s] > 0)
-                    mbar_wait(smem_u32(&q_full[s]), (qcount[s] - 1) & 1, p.timeout_ns, nullptr);
-        }
-    } else if (warp == 1) {
-        // ================================================= MMA issuer
-        if (lane == 0) {
-            const uint32_t idS = idesc_f16(kBF16, 128, 128, false);
-            const uint32_t idO = idesc_f16(kBF16, 128, p.d, true);
-            const int nk = p.d / 16;
-            const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
-            const uint64_t dK0 = smem_desc_sw128(sRing, 16, 1024);
-            const uint64_t dV0 = smem_desc_sw128(sRing, kChunkBytes, 1024);
-            uint32_t qcount[2] = {0, 0};   // units started per slot
-            uint32_t pcount[2] = {0, 0};   // tiles whose P was consumed, per slot
-            int64_t li = 0;                // K/V loads consumed (ring position)
-            bool ok = true;
-            for (int pass = 0; ok; ++pass) {
-                const int unit = prefill_pass_unit(pass);
-                if (unit >= n_units) break;
-                int b, kvh;
-                SlotInfo slot[2];
-                prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
-                const int nmax = max(slot[0].n_kv, slot[1].n_kv);
-                const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
-                                 : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    if (slot[s].n_kv == 0 || !ok) continue;
-                    ok = mbar_wait(smem_u32(&q_full[s]), qcount[s] & 1, p.timeout_ns, abort_flag);
-                    ++qcount[s];
-                }
-                if (ok) ok = mbar_wait(smem_u32(&kv_full[li % NST]), uint32_t((li / NST) & 1), p.timeout_ns,
-                                       abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                {
-                    const int stK = int(li % NST);
-#pragma unroll
+    if (warp < 4) {
+        reg_dealloc<kPfRegsLow>();
+        if (warp == 0) {
+            // ================================================= TMA producer
+            if (lane == 0) {
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmV);
+                uint32_t qcount[2] = {0, 0};   // Q loads per slot so far
+                int64_t li = 0;                // K/V loads so far (ring position)
+                bool ok = true;
+                for (int pass = 0; ok; ++pass) {
+                    const int unit = prefill_pass_unit(pass);
+                    if (unit >= n_units) break;
+                    int b, kvh;
+                    SlotInfo slot[2];
+                    prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                    const int nmax = max(slot[0].n_kv, slot[1].n_kv);
+                    const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
+                                     : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
+    #pragma unroll
                     for (int s = 0; s < 2; ++s) {
-                        if (slot[s].n_kv == 0 || slot[s].n_lo != nmin) continue;
-                        issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
-                        mma_commit(smem_u32(&s_full[s]));
-                        if (nmin + 1 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
+                        if (slot[s].n_kv == 0) continue;
+                        // the previous unit's Q.K^T MMAs of this slot are done with Q
+                        if (qcount[s] > 0 &&
+                            !mbar_wait(smem_u32(&q_empty[s]), (qcount[s] - 1) & 1, p.timeout_ns, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t bar = smem_u32(&q_full[s]);
+                        mbar_expect_tx(bar, DCH * kChunkBytes);
+                        for (int c = 0; c < DCH; ++c)
+                            tma_load_3d(sQ + (s * DCH + c) * kChunkBytes, &tmQ, bar, c * 64, slot[s].q0,
+                                        b * p.H + slot[s].h);
+                        ++qcount[s];
                     }
-                    mma_commit(smem_u32(&kv_empty[stK]));
-                    ++li;
+                    const int zkv = b * p.Hkv + kvh;
+                    const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * (nmax - nmin);
+                    for (int i = 0; i < n_loads && ok; ++i, ++li) {
+                        const int st = int(li % NST);
+                        if (!mbar_wait(smem_u32(&kv_empty[st]), uint32_t((li / NST) & 1) ^ 1, p.timeout_ns,
+                                       abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t bar = smem_u32(&kv_full[st]);
+                        mbar_expect_tx(bar, DCH * kChunkBytes);
+                        const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+                        if (PAGED)
+                            load_kv_paged<DCH>(p, sRing + st * DCH * kChunkBytes, map, bar, nmin + (i >> 1), b,
+                                               kvh, slot[0].S);
+                        else
+                            for (int c = 0; c < DCH; ++c)
+                                tma_load_3d(sRing + (st * DCH + c) * kChunkBytes, map, bar, c * 64,
+                                            (nmin + (i >> 1)) * 128, zkv);
+                    }
                 }
-                for (int n = nmin; n < nmax && ok; ++n) {
-                    const int64_t iV = li, iK = li + 1;
-                    const int stV = int(iV % NST), stK = int(iK % NST);
-                    const bool nextK = n + 1 < nmax;
-                    ok = mbar_wait(smem_u32(&kv_full[stV]), uint32_t((iV / NST) & 1), p.timeout_ns, abort_flag);
-                    if (ok && nextK)
-                        ok = mbar_wait(smem_u32(&kv_full[stK]), uint32_t((iK / NST) & 1), p.timeout_ns,
-                                       abort_flag);
+                // no copy may still be landing in shared memory when the CTA exits
+                for (int64_t i = li - 1; i >= 0 && i >= li - NST; --i)
+                    mbar_wait(smem_u32(&kv_full[i % NST]), uint32_t((i / NST) & 1), p.timeout_ns, nullptr);
+                for (int s = 0; s < 2; ++s)
+                    if (qcount[s] > 0)
+                        mbar_wait(smem_u32(&q_full[s]), (qcount[s] - 1) & 1, p.timeout_ns, nullptr);
+            }
+        } else if (warp == 1) {
+            // ================================================= MMA issuer
+            if (lane == 0) {
+                const uint32_t idS = idesc_f16(kBF16, 128, 128, false);
+                const uint32_t idO = idesc_f16(kBF16, 128, p.d, true);
+                const int nk = p.d / 16;
+                const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
+                const uint64_t dK0 = smem_desc_sw128(sRing, 16, 1024);
+                const uint64_t dV0 = smem_desc_sw128(sRing, kChunkBytes, 1024);
+                uint32_t qcount[2] = {0, 0};   // units started per slot
+                uint32_t pcount[2] = {0, 0};   // tiles whose P was consumed, per slot
+                int64_t li = 0;                // K/V loads consumed (ring position)
+                bool ok = true;
+                for (int pass = 0; ok; ++pass) {
+                    const int unit = prefill_pass_unit(pass);
+                    if (unit >= n_units) break;
+                    int b, kvh;
+                    SlotInfo slot[2];
+                    prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                    const int nmax = max(slot[0].n_kv, slot[1].n_kv);
+                    const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
+                                     : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
+    #pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        if (slot[s].n_kv == 0 || !ok) continue;
+                        ok = mbar_wait(smem_u32(&q_full[s]), qcount[s] & 1, p.timeout_ns, abort_flag);
+                        ++qcount[s];
+                    }
+                    if (ok) ok = mbar_wait(smem_u32(&kv_full[li % NST]), uint32_t((li / NST) & 1), p.timeout_ns,
+                                           abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int s = 0; s < 2; ++s) {
-                        // a slot whose window starts at tile n + 1 only gets its first S here
-                        const bool first_next = WINDOW && n + 1 == slot[s].n_lo && n + 1 < slot[s].n_kv;
-                        if (first_next) {
+                    {
+                        const int stK = int(li % NST);
+    #pragma unroll
+                        for (int s = 0; s < 2; ++s) {
+                            if (slot[s].n_kv == 0 || slot[s].n_lo != nmin) continue;
                             issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
                             mma_commit(smem_u32(&s_full[s]));
-                            if (n + 2 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
+                            if (nmin + 1 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
                         }
-                        if (!ok || n < slot[s].n_lo || n >= slot[s].n_kv) continue;
-                        const uint32_t par = pcount[s] & 1;
-                        // P in two halves: the first 64 keys' MMAs start while the
-                        // softmax is still producing the second half
-                        if (!mbar_wait(smem_u32(&p_ready[2 * s]), par, p.timeout_ns, abort_flag)) {
-                            ok = false;
-                            continue;
-                        }
-                        tc_fence_after();
-                        issue_PV<0, DCH>(dV0, tmem, idO, s, stV, n > slot[s].n_lo);
-                        if (!mbar_wait(smem_u32(&p_ready[2 * s + 1]), par, p.timeout_ns, abort_flag)) {
-                            ok = false;
-                            continue;
-                        }
-                        tc_fence_after();
-                        issue_PV<4, DCH>(dV0, tmem, idO, s, stV, true);
-                        ++pcount[s];
-                        if (n == slot[s].n_kv - 1) mma_commit(smem_u32(&o_done[s]));
-                        if (n + 1 < slot[s].n_kv) {
-                            issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
-                            mma_commit(smem_u32(&s_full[s]));
-                            if (n + 2 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
-                        }
-                    }
-                    if (!ok) break;
-                    mma_commit(smem_u32(&kv_empty[stV]));
-                    ++li;
-                    if (nextK) {
                         mma_commit(smem_u32(&kv_empty[stK]));
                         ++li;
                     }
+                    for (int n = nmin; n < nmax && ok; ++n) {
+                        const int64_t iV = li, iK = li + 1;
+                        const int stV = int(iV % NST), stK = int(iK % NST);
+                        const bool nextK = n + 1 < nmax;
+                        ok = mbar_wait(smem_u32(&kv_full[stV]), uint32_t((iV / NST) & 1), p.timeout_ns, abort_flag);
+                        if (ok && nextK)
+                            ok = mbar_wait(smem_u32(&kv_full[stK]), uint32_t((iK / NST) & 1), p.timeout_ns,
+                                           abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+    #pragma unroll
+                        for (int s = 0; s < 2; ++s) {
+                            // a slot whose window starts at tile n + 1 only gets its first S here
+                            const bool first_next = WINDOW && n + 1 == slot[s].n_lo && n + 1 < slot[s].n_kv;
+                            if (first_next) {
+                                issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
+                                mma_commit(smem_u32(&s_full[s]));
+                                if (n + 2 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
+                            }
+                            if (!ok || n < slot[s].n_lo || n >= slot[s].n_kv) continue;
+                            const uint32_t par = pcount[s] & 1;
+                            // P in two halves: the first 64 keys' MMAs start while the
+                            // softmax is still producing the second half
+                            if (!mbar_wait(smem_u32(&p_ready[2 * s]), par, p.timeout_ns, abort_flag)) {
+                                ok = false;
+                                continue;
+                            }
+                            tc_fence_after();
+                            issue_PV<0, DCH>(dV0, tmem, idO, s, stV, n > slot[s].n_lo);
+                            if (!mbar_wait(smem_u32(&p_ready[2 * s + 1]), par, p.timeout_ns, abort_flag)) {
+                                ok = false;
+                                continue;
+                            }
+                            tc_fence_after();
+                            issue_PV<4, DCH>(dV0, tmem, idO, s, stV, true);
+                            ++pcount[s];
+                            if (n == slot[s].n_kv - 1) mma_commit(smem_u32(&o_done[s]));
+                            if (n + 1 < slot[s].n_kv) {
+                                issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
+                                mma_commit(smem_u32(&s_full[s]));
+                                if (n + 2 == slot[s].n_kv) mma_commit(smem_u32(&q_empty[s]));
+                            }
+                        }
+                        if (!ok) break;
+                        mma_commit(smem_u32(&kv_empty[stV]));
+                        ++li;
+                        if (nextK) {
+                            mma_commit(smem_u32(&kv_empty[stK]));
+                            ++li;
+                        }
+                    }
                 }
+                // every MMA issued must finish before TMEM is released
+                mma_commit(smem_u32(drain));
+                mbar_wait(smem_u32(drain), 0, p.timeout_ns, nullptr);
             }
-            // every MMA issued must finish before TMEM is released
-            mma_commit(smem_u32(drain));
-            mbar_wait(smem_u32(drain), 0, p.timeout_ns, nullptr);
         }
-    } else if (warp >= 4) {
+    } else {
+        reg_alloc<kPfRegsHigh>();
         // ================================================= softmax + epilogue
         // warps 4-7: slot 0, warps 8-11: slot 1; one thread per row (TMEM lane).
         const int s = (warp - 4) >> 2;

@@ -94,6 +94,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     }
 }
 
+// ------------------------------------------------------------------ registers
+
+// Per-warpgroup register limits (setmaxnreg): every warp of a warpgroup
+// executes the same call.  An increase waits until the block's own pool (its
+// threads x the registers per thread at launch) can cover it, so a split
+// must fit that pool; the host checks it before the first launch.
+template <int N> __device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N> __device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
