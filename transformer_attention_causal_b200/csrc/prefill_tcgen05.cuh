@@ -369,7 +369,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                     const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                      : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
-    #pragma unroll
+#pragma unroll
                     for (int s = 0; s < 2; ++s) {
                         if (slot[s].n_kv == 0) continue;
                         // the previous unit's Q.K^T MMAs of this slot are done with Q
@@ -435,7 +435,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                     const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                      : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
-    #pragma unroll
+#pragma unroll
                     for (int s = 0; s < 2; ++s) {
                         if (slot[s].n_kv == 0 || !ok) continue;
                         ok = mbar_wait(smem_u32(&q_full[s]), qcount[s] & 1, p.timeout_ns, abort_flag);
@@ -447,7 +447,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     tc_fence_after();
                     {
                         const int stK = int(li % NST);
-    #pragma unroll
+#pragma unroll
                         for (int s = 0; s < 2; ++s) {
                             if (slot[s].n_kv == 0 || slot[s].n_lo != nmin) continue;
                             issue_S<DCH>(dQ0, dK0, tmem, idS, nk, s, stK);
@@ -467,7 +467,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                                            abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-    #pragma unroll
+#pragma unroll
                         for (int s = 0; s < 2; ++s) {
                             // a slot whose window starts at tile n + 1 only gets its first S here
                             const bool first_next = WINDOW && n + 1 == slot[s].n_lo && n + 1 < slot[s].n_kv;
