@@ -212,8 +212,9 @@ ATTN_API size_t attn_cached_local_workspace_size(attn_dtype_t dtype, int64_t B, 
  *     aligned; may be NULL when that size is 0.
  * The device arrays are read, never written; entries out of range are
  * reported through attn_device_status() as ATTN_ERR_DEVICE_INDEX.
- * Kernels: bf16 / fp16 with d in {64, 128} and H / Hkv * Tnew <= 16, or
- * d = 256 and H / Hkv * Tnew <= 8, run the split-KV decode kernels; other
+ * Kernels: bf16 / fp16 with d a multiple of 16 in [64, 128] and
+ * H / Hkv * Tnew <= 16, or d = 256 and H / Hkv * Tnew <= 8, run the split-KV
+ * decode kernels; other
  * bf16 / fp16 shapes with d a multiple of 16 in [64, 128] (chunked prefill)
  * run the tensor-core prefill kernel, which copies whole pages: there the
  * rows of a sequence's last page past L_b are read (with zero weight) and

@@ -133,6 +133,10 @@ def test_plans_pick_the_intended_kernels(lib):
     assert lib.attn_prefill_plan(BF16, 1, 32, 32, 2048, 80, 1) == L.KERNEL_TCGEN05
     assert lib.attn_prefill_plan(BF16, 8, 16, 8, 4096, 128, 1) == L.KERNEL_TCGEN05
     assert lib.attn_cached_plan(BF16, 64, 32, 8, 1, 8192, 8192, 128, 8191) == L.KERNEL_SPLITKV
+    # decode at every tensor-core head size (BitNet-3B: MHA, d = 80)
+    for d in (64, 80, 96, 112):
+        assert lib.attn_cached_plan(BF16, 1, 32, 32, 1, 2048, 2048, d, 2047) == L.KERNEL_SPLITKV
+    assert lib.attn_cached_plan(BF16, 1, 32, 32, 17, 2048, 2048, 80, 2031) == L.KERNEL_TCGEN05
     assert lib.attn_cached_plan(F16, 32, 8, 1, 512, 4096, 4096, 128, 3584) == L.KERNEL_TCGEN05
     # head sizes the tensor-core kernel does not take fall back to CUDA cores
     assert lib.attn_prefill_plan(BF16, 1, 2, 1, 16, 40, 1) == L.KERNEL_SIMT

@@ -79,6 +79,8 @@ CASES = [
     (2, 16, 4, 4, 128, [700, 1500], 256, F16),         # 4 new tokens per sequence
     (2, 8, 1, 1, 64, [333, 64], 8, BF16),              # MQA, d = 64, the smallest pages
     (2, 4, 4, 2, 256, [900, 129], 32, F16),            # d = 256
+    (3, 8, 8, 1, 80, [700, 129, 2048], 64, BF16),      # MHA decode, d = 80
+    (2, 8, 2, 2, 96, [333, 1000], 16, F16),            # d = 96, 8 rows per K/V head
     (4, 8, 8, 1, 128, [1, 5, 128, 129], 128, BF16),    # lengths at page edges, a single token
     # chunked prefill (many new rows per K/V head): the tensor-core kernel
     # copying whole pages, one to sixteen copies per 128-key tile

@@ -152,6 +152,10 @@ CACHED_CASES = [
     (BF16, 1, 4, 1, 1, 19999, 20000, 20000, 128, "splitkv"),  # one long sequence: many splits
     (BF16, 2, 4, 2, 1, 0, 1, 1, 128, "splitkv"),            # first token
     (F16, 2, 16, 1, 1, 1999, 2000, 2048, 64, "splitkv"),    # 16 rows per K/V head at d = 64
+    (BF16, 2, 8, 8, 1, 1299, 1300, 1300, 80, "splitkv"),    # MHA decode, d = 80 (a part-filled chunk)
+    (F16, 1, 8, 2, 3, 997, 1000, 1024, 96, "splitkv"),      # d = 96, 12 rows per K/V head
+    (BF16, 2, 16, 2, 1, 2047, 2048, 2048, 112, "splitkv"),  # d = 112, 8 rows
+    (BF16, 1, 4, 1, 4, 4999, 5003, 5003, 80, "splitkv"),    # d = 80, 16 rows, several splits
     (F16, 2, 8, 1, 200, 300, 500, 520, 128, "tcgen05"),     # MQA chunked prefill
     (BF16, 1, 4, 2, 64, 37, 101, 101, 80, "tcgen05"),       # unaligned start
     (BF16, 1, 2, 2, 100, 400, 600, 640, 64, "tcgen05"),     # history past the last query

@@ -86,6 +86,8 @@ CACHED = [
     (BF16, 2, 32, 8, 1, 8191, 8192, 128, 1024, "splitkv"),   # GQA decode, several splits
     (F16, 2, 4, 1, 4, 3000, 3004, 128, 100, "splitkv"),      # 4 new tokens: per-row edges
     (BF16, 1, 4, 4, 2, 2000, 2002, 256, 700, "splitkv"),     # d = 256
+    (BF16, 2, 8, 8, 1, 3000, 3001, 80, 500, "splitkv"),      # MHA decode, d = 80
+    (F16, 1, 8, 2, 2, 1500, 1502, 112, 129, "splitkv"),      # d = 112, per-row edges
     (F16, 2, 8, 1, 200, 300, 500, 128, 64, "tcgen05"),       # chunked prefill with a window
     (F32, 1, 4, 2, 5, 60, 70, 32, 9, "simt"),
 ]

@@ -75,7 +75,7 @@ attn_status_t check_shape(const Problem& pb) {
 }
 
 int decode_rmax(int64_t d) {
-    if (d == 64 || d == 128) return 16;
+    if (d % 16 == 0 && d >= 64 && d <= 128) return 16;
     if (d == 256) return 8;
     return 0;
 }
@@ -91,9 +91,9 @@ void plan_decode(const Problem& pb, Plan& pl) {
     const int64_t G = pb.H / pb.Hkv;
     pl.Rv = int(G * pb.Tq);
     pl.R = next_pow2_at_least4(pl.Rv);
-    // d = 64 / 128: the MMA kernel (128-key stages, one CTA per SM); d = 256:
-    // the CUDA-core kernel (64-key stages, two CTAs per SM)
-    pl.mma = (pb.d == 64 || pb.d == 128) && pl.Rv <= 16;
+    // d a multiple of 16 in [64, 128]: the MMA kernel (128-key stages, one CTA
+    // per SM); d = 256: the CUDA-core kernel (64-key stages, two CTAs per SM)
+    pl.mma = pb.d % 16 == 0 && pb.d >= 64 && pb.d <= 128 && pl.Rv <= 16;
     const int stage_keys = pl.mma ? kDecMmaTK : 64;
     const int ctas_per_sm = pl.mma ? 1 : 2;
     pl.kv_end = std::min<int64_t>(pb.S, pb.start_pos + pb.Tq);
@@ -286,11 +286,11 @@ attn_status_t launch_decode_256(int R, const DecodeParams& dp, cudaStream_t stre
     }
 }
 
-template <typename T, int DCH, int NT, bool WINDOW, bool PAGED = false>
+template <typename T, int D, int NT, bool WINDOW, bool PAGED = false>
 attn_status_t launch_decode_mma_k(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& dp,
                                   cudaStream_t stream) {
-    constexpr size_t smem = DecMmaShape<DCH>::smem_bytes();
-    auto kern = decode_mma_kernel<T, DCH, NT, WINDOW, PAGED>;
+    constexpr size_t smem = DecMmaShape<(D + 63) / 64>::smem_bytes();
+    auto kern = decode_mma_kernel<T, D, NT, WINDOW, PAGED>;
     static std::once_flag once[8];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -302,10 +302,25 @@ attn_status_t launch_decode_mma_k(const CUtensorMap& mk, const CUtensorMap& mv, 
     if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
     if (dp.nsplit > 1) {
         const int64_t rows = int64_t(dp.B) * dp.Hkv * dp.Rv;
-        decode_combine_kernel<T, 64 * DCH><<<unsigned((rows + 3) / 4), 128, 0, stream>>>(dp);
+        decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, stream>>>(dp);
         return launch_status();
     }
     return ATTN_OK;
+}
+
+// One head size: rows padded to 8 or 16; plain, windowed or paged cache.
+template <typename T, int D>
+attn_status_t launch_decode_mma_d(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& dp,
+                                  cudaStream_t stream) {
+    const bool two = dp.Rv > 8;
+    if (dp.paged)
+        return two ? launch_decode_mma_k<T, D, 2, false, true>(mk, mv, dp, stream)
+                   : launch_decode_mma_k<T, D, 1, false, true>(mk, mv, dp, stream);
+    if (dp.window > 0)
+        return two ? launch_decode_mma_k<T, D, 2, true>(mk, mv, dp, stream)
+                   : launch_decode_mma_k<T, D, 1, true>(mk, mv, dp, stream);
+    return two ? launch_decode_mma_k<T, D, 2, false>(mk, mv, dp, stream)
+               : launch_decode_mma_k<T, D, 1, false>(mk, mv, dp, stream);
 }
 
 template <typename T>
@@ -319,26 +334,18 @@ attn_status_t launch_decode_mma(const Problem& pb, const DecodeParams& dp, cudaS
         if (encode_rows(&mk, dp.k, pb.dt, pb.d, page_size, page_size, dp.num_pages * pb.Hkv, rows) != ATTN_OK ||
             encode_rows(&mv, dp.v, pb.dt, pb.d, page_size, page_size, dp.num_pages * pb.Hkv, rows) != ATTN_OK)
             return ATTN_ERR_CUDA;
-        if (pb.d == 64)
-            return dp.Rv > 8 ? launch_decode_mma_k<T, 1, 2, false, true>(mk, mv, dp, stream)
-                             : launch_decode_mma_k<T, 1, 1, false, true>(mk, mv, dp, stream);
-        return dp.Rv > 8 ? launch_decode_mma_k<T, 2, 2, false, true>(mk, mv, dp, stream)
-                         : launch_decode_mma_k<T, 2, 1, false, true>(mk, mv, dp, stream);
-    }
-    if (encode_rows(&mk, dp.k, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK ||
-        encode_rows(&mv, dp.v, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK)
+    } else if (encode_rows(&mk, dp.k, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK ||
+               encode_rows(&mv, dp.v, pb.dt, pb.d, pb.S, pb.S_cap, pb.B * pb.Hkv) != ATTN_OK) {
         return ATTN_ERR_CUDA;
-    const bool two = dp.Rv > 8, win = dp.window > 0;
-    if (pb.d == 64) {
-        if (two) return win ? launch_decode_mma_k<T, 1, 2, true>(mk, mv, dp, stream)
-                            : launch_decode_mma_k<T, 1, 2, false>(mk, mv, dp, stream);
-        return win ? launch_decode_mma_k<T, 1, 1, true>(mk, mv, dp, stream)
-                   : launch_decode_mma_k<T, 1, 1, false>(mk, mv, dp, stream);
     }
-    if (two) return win ? launch_decode_mma_k<T, 2, 2, true>(mk, mv, dp, stream)
-                        : launch_decode_mma_k<T, 2, 2, false>(mk, mv, dp, stream);
-    return win ? launch_decode_mma_k<T, 2, 1, true>(mk, mv, dp, stream)
-               : launch_decode_mma_k<T, 2, 1, false>(mk, mv, dp, stream);
+    switch (pb.d) {
+    case 64: return launch_decode_mma_d<T, 64>(mk, mv, dp, stream);
+    case 80: return launch_decode_mma_d<T, 80>(mk, mv, dp, stream);
+    case 96: return launch_decode_mma_d<T, 96>(mk, mv, dp, stream);
+    case 112: return launch_decode_mma_d<T, 112>(mk, mv, dp, stream);
+    case 128: return launch_decode_mma_d<T, 128>(mk, mv, dp, stream);
+    default: return ATTN_ERR_UNSUPPORTED;
+    }
 }
 
 // A paged K/V cache: page pools, the page table and the per-sequence lengths.

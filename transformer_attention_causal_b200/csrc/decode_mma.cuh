@@ -1,7 +1,7 @@
-// Split-KV cached decode on warp-level tensor-core MMAs (contiguous cache,
-// d = 64 or 128, up to 16 rows per K/V head).
+// Split-KV cached decode on warp-level tensor-core MMAs (d a multiple of 16
+// in [64, 128], up to 16 rows per K/V head; contiguous or paged cache).
 //
-// Same split, online softmax and merge as decode_wide_kernel ("Multi-query
+// Same split, online softmax and merge as decode_splitkv_kernel ("Multi-query
 // attention, annotated" §2.4.1: the call streams the visible history once,
 // so it is bound by HBM), with the per-key arithmetic moved off the FMA pipes:
 // the CUDA-core kernels spend ~64 warp instructions per key on widening,
@@ -20,7 +20,9 @@
 //   O^T (d x 8 rows) += V^T P^T       mma.m16n8k16 with V^T from ldmatrix.trans.
 // About four instructions per key.  K and V stages arrive by TMA with the
 // 128-byte swizzle (conflict-free ldmatrix rows); rows past the end of the
-// history are zero-filled by TMA and masked by position.
+// history are zero-filled by TMA and masked by position.  A head size that is
+// not a multiple of 64 fills its last 64-column chunk partly (TMA zero-fills
+// the rest) and runs d / 16 k-steps and m-tiles.
 // Paged variant: each 128-key stage is one TMA copy per page it spans (boxes
 // of min(P, 128) rows over the pools); rows past the sequence's end and
 // out-of-range page ids (reported) are read at an out-of-range coordinate and
@@ -50,11 +52,12 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t tile, int key, int d0) {
     return tile + uint32_t(d0 >> 6) * 16384u + uint32_t(key) * 128u + (uint32_t(u ^ (key & 7)) << 4);
 }
 
-template <typename T, int DCH, int NT, bool WINDOW, bool PAGED>
+template <typename T, int D, int NT, bool WINDOW, bool PAGED>
 __global__ void __launch_bounds__(kDecMmaThreads, 1)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeParams p) {
-    constexpr int D = 64 * DCH;
+    static_assert(D % 16 == 0 && D >= 64 && D <= 128, "head size");
+    constexpr int DCH = (D + 63) / 64;          // 64-column chunks of a K/V row
     constexpr int NK = D / 16;                  // k-steps of S^T, m-tiles of O^T
     constexpr int NW = kDecMmaWarps, TK = kDecMmaTK;
     constexpr int NST = DecMmaShape<DCH>::NST;
