@@ -215,6 +215,32 @@ attn_status_t set_smem(K kernel, size_t bytes) {
                : ATTN_ERR_CUDA;
 }
 
+constexpr int kMaxDevices = 64;
+
+// Once per kernel and device: its dynamic shared-memory limit and, for a
+// kernel that moves registers between warpgroups (setmaxnreg), a check that
+// its launch allocation (threads x registers) covers `regs_needed`, since an
+// increase the block's pool cannot grant never returns.  The outcome is kept
+// and returned on every later call, so a failure is never followed by a
+// launch.
+template <auto Kern>
+attn_status_t prepare_kernel(size_t smem, int threads = 0, int regs_needed = 0) {
+    static std::once_flag once[kMaxDevices];
+    static attn_status_t status[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    std::call_once(once[dev], [&] {
+        attn_status_t r = set_smem(Kern, smem);
+        if (r == ATTN_OK && regs_needed > 0) {
+            cudaFuncAttributes fa{};
+            if (cudaFuncGetAttributes(&fa, Kern) != cudaSuccess || fa.numRegs * threads < regs_needed)
+                r = ATTN_ERR_CUDA;
+        }
+        status[dev] = r;
+    });
+    return status[dev];
+}
+
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count() {
     static std::atomic<int> cached[64];
@@ -251,13 +277,8 @@ attn_status_t run_simt(const Problem& pb, const void* q, const void* k, const vo
 template <typename T, int D, int R, int MODE>
 attn_status_t launch_decode_RP(const DecodeParams& dp, cudaStream_t stream) {
     constexpr size_t smem = DecodeShape<D, R>::smem_bytes(sizeof(T));
-    auto kern = decode_splitkv_kernel<T, D, R, MODE>;
-    static std::once_flag once[8];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    attn_status_t st = ATTN_OK;
-    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
-    if (st != ATTN_OK) return st;
+    constexpr auto kern = &decode_splitkv_kernel<T, D, R, MODE>;
+    if (const attn_status_t st = prepare_kernel<kern>(smem); st != ATTN_OK) return st;
     dim3 grid(unsigned(dp.nsplit), unsigned(dp.B * dp.Hkv));
     kern<<<grid, 160, smem, stream>>>(dp);
     if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
@@ -290,13 +311,8 @@ template <typename T, int D, int NT, bool WINDOW, bool PAGED = false>
 attn_status_t launch_decode_mma_k(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& dp,
                                   cudaStream_t stream) {
     constexpr size_t smem = DecMmaShape<(D + 63) / 64>::smem_bytes();
-    auto kern = decode_mma_kernel<T, D, NT, WINDOW, PAGED>;
-    static std::once_flag once[8];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    attn_status_t st = ATTN_OK;
-    std::call_once(once[dev & 7], [&] { st = set_smem(kern, smem); });
-    if (st != ATTN_OK) return st;
+    constexpr auto kern = &decode_mma_kernel<T, D, NT, WINDOW, PAGED>;
+    if (const attn_status_t st = prepare_kernel<kern>(smem); st != ATTN_OK) return st;
     dim3 grid(unsigned(dp.nsplit), unsigned(dp.B * dp.Hkv));
     kern<<<grid, kDecMmaThreads, smem, stream>>>(mk, mv, dp);
     if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
@@ -393,21 +409,12 @@ attn_status_t launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk
                                     const CUtensorMap& mv, const PrefillParams& pp, int64_t grid,
                                     cudaStream_t stream) {
     constexpr size_t smem = prefill_smem_bytes<DCH>();
-    auto kern = prefill_tcgen05_kernel<T, DCH, WINDOW, PAGED>;
-    static std::once_flag once[8];
-    static attn_status_t ready[8];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    std::call_once(once[dev & 7], [&] {
-        attn_status_t r = set_smem(kern, smem);
-        // the kernel's register split must fit the block's launch allocation,
-        // or its increase would never be granted
-        cudaFuncAttributes fa{};
-        if (r == ATTN_OK && cudaFuncGetAttributes(&fa, kern) != cudaSuccess) r = ATTN_ERR_CUDA;
-        if (r == ATTN_OK && fa.numRegs * kPfThreads < 128 * kPfRegsLow + 256 * kPfRegsHigh) r = ATTN_ERR_CUDA;
-        ready[dev & 7] = r;
-    });
-    if (ready[dev & 7] != ATTN_OK) return ready[dev & 7];
+    constexpr auto kern = &prefill_tcgen05_kernel<T, DCH, WINDOW, PAGED>;
+    // the register split: warpgroup 0 at kPfRegsLow, the two softmax warpgroups at kPfRegsHigh
+    if (const attn_status_t st =
+            prepare_kernel<kern>(smem, kPfThreads, 128 * kPfRegsLow + 256 * kPfRegsHigh);
+        st != ATTN_OK)
+        return st;
     kern<<<unsigned(grid), kPfThreads, smem, stream>>>(mq, mk, mv, pp);
     return launch_status();
 }
@@ -586,15 +593,6 @@ size_t backward_ws_bytes(const Problem& pb) {
     return (bytes + 255) & ~size_t(255);
 }
 
-template <typename K>
-attn_status_t set_smem_once(K kern, size_t bytes, std::once_flag (&once)[8]) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    attn_status_t st = ATTN_OK;
-    std::call_once(once[dev & 7], [&] { st = set_smem(kern, bytes); });
-    return st;
-}
-
 template <typename T, int DCH, bool WINDOW>
 attn_status_t launch_backward(const Problem& pb, BwdParams& bp, const void* q, const void* k,
                               const void* v, const void* dout, cudaStream_t stream) {
@@ -610,13 +608,11 @@ attn_status_t launch_backward(const Problem& pb, BwdParams& bp, const void* q, c
     bwd_preprocess_kernel<T><<<unsigned(pre_blocks), 256, 0, stream>>>(bp);
     if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
 
-    static std::once_flag once_kv[8], once_q[8];
     constexpr size_t smem_kv = bwd_dkdv_smem_bytes<DCH>();
     constexpr size_t smem_q = bwd_dq_smem_bytes<DCH>();
-    auto kern_kv = bwd_dkdv_kernel<T, DCH, WINDOW>;
-    auto kern_q = bwd_dq_kernel<T, DCH, WINDOW>;
-    if (set_smem_once(kern_kv, smem_kv, once_kv) != ATTN_OK ||
-        set_smem_once(kern_q, smem_q, once_q) != ATTN_OK)
+    constexpr auto kern_kv = &bwd_dkdv_kernel<T, DCH, WINDOW>;
+    constexpr auto kern_q = &bwd_dq_kernel<T, DCH, WINDOW>;
+    if (prepare_kernel<kern_kv>(smem_kv) != ATTN_OK || prepare_kernel<kern_q>(smem_q) != ATTN_OK)
         return ATTN_ERR_CUDA;
     kern_kv<<<unsigned(int64_t(bp.n_t) * bp.B * bp.Hkv), kBwdThreads, smem_kv, stream>>>(mq, mk, mv,
                                                                                         mdo, bp);
