@@ -102,10 +102,15 @@ void plan_decode(const Problem& pb, Plan& pl) {
     const int64_t tiles = (pl.kv_end - pl.k_lo + stage_keys - 1) / stage_keys;
     const int64_t units = pb.B * pb.Hkv;
     const int64_t slots = int64_t(kPlanSMs) * ctas_per_sm;
-    // Pick the split count that fills the last wave of CTAs best; prefer fewer
-    // splits on ties and keep at least 4 stages per split when there is room.
+    // Pick the split count with the least modelled time: waves of CTAs, each
+    // costing its stages plus a start-up and merge worth about three stages
+    // (one CTA per SM, so a wave's start is not hidden behind the last one's
+    // stages); fewer splits on ties, at least 4 stages per split when there
+    // is room.  Against filling the last wave best, this halves the CTAs of
+    // mid-size calls (B = 8, S = 8192: 3.0 -> 3.9 TB/s at d = 96, 3.5 -> 4.3
+    // at d = 128) and leaves the large ones as they were.
     int best_n = 1;
-    double best_score = -1.0;
+    double best_score = -1e300;
     const int64_t max_n = std::max<int64_t>(1, std::min<int64_t>(tiles, 128));
     for (int64_t n = 1; n <= max_n; ++n) {
         const int64_t per = (tiles + n - 1) / n;
@@ -114,8 +119,7 @@ void plan_decode(const Problem& pb, Plan& pl) {
         if (per < 4 && n > 1 && units * (n - 1) >= slots) continue;
         const int64_t ctas = units * n;
         const int64_t waves = (ctas + slots - 1) / slots;
-        const double fill = double(ctas) / double(waves * slots);
-        const double score = fill - 0.002 * double(n);
+        const double score = -double(waves) * (3.0 + double(per)) - 1e-3 * double(n);
         if (score > best_score + 1e-12) {
             best_score = score;
             best_n = int(n);
