@@ -153,6 +153,27 @@ def test_workspace_size_is_zero_without_splits(lib):
     assert lib.attn_cached_workspace_size(BF16, 1, 4, 3, 1, 64, 128, 63) == 0
 
 
+def test_split_counts_of_the_decode_planner(lib):
+    """The split count, read back from the workspace size (fp32 partials:
+    units x splits x rows x (d + 2) floats, rounded up to 256 bytes).  The
+    planner models a call as waves of CTAs over 148 SMs, each CTA costing
+    its 128-key stages plus about three stages of start-up and merge."""
+    def splits(B, H, Hkv, S, d):
+        ws = lib.attn_cached_workspace_size(BF16, B, H, Hkv, 1, S, d, S - 1)
+        per_split = B * Hkv * (H // Hkv) * (d + 2) * 4
+        n = ws // per_split
+        assert ws == 0 or (ws - n * per_split) < 256
+        return max(n, 1)
+    # GQA decode, 512 units of 64 stages: 2 splits (7 waves of 32-stage CTAs)
+    assert splits(64, 32, 8, 8192, 128) == 2
+    # 64 units: one wave of 128 CTAs beats 7 waves of 4-stage CTAs
+    assert splits(8, 32, 8, 8192, 128) == 2
+    # MHA d = 80, 256 units of 32 stages: no split (two waves)
+    assert splits(8, 32, 32, 4096, 80) == 1
+    # one sequence on one K/V head, 157 stages: 79 splits of 2 (one wave)
+    assert splits(1, 4, 1, 20000, 128) == 79
+
+
 def append(lib, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, dt=BF16, B=1, Hkv=2, Tnew=4, S_cap=16, d=64,
            start_pos=3, base=10000.0):
     return lib.attn_kv_append_rope(k, v, kc, vc, dt, B, Hkv, Tnew, S_cap, d, start_pos, base, None)
