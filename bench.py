@@ -379,9 +379,27 @@ class Case:
                              workspace=self.ws, stream=stream)
 
 
+# per-call device times (ms) of the latest time_device() call on this rank
+_LAST_CALL_MS: list = []
+
+
+def spread(times_ms):
+    """Median and 10th / 90th percentiles (nearest rank) of per-call times."""
+    t = sorted(times_ms)
+    if not t:
+        return None
+
+    def pick(q):
+        return t[min(len(t) - 1, max(0, math.ceil(q * len(t)) - 1))]
+
+    return {"median_ms": round(statistics.median(t), 5), "p10_ms": round(pick(0.10), 5),
+            "p90_ms": round(pick(0.90), 5)}
+
+
 def time_device(case, steps, warmup, dist_ctx):
     """Mean per-call device time (ms) over `steps` timed calls, L2 flushed
-    before each; returns (kernel_ms, bracket_ms)."""
+    before each; returns (kernel_ms, bracket_ms).  The per-call times are
+    left in _LAST_CALL_MS."""
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=case.device)
     for _ in range(warmup):
         flush.zero_()
@@ -401,7 +419,9 @@ def time_device(case, steps, warmup, dist_ctx):
     b1.record()
     torch.cuda.synchronize()
     dist_ctx.barrier()
-    kernel_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(steps)) / steps
+    times = [ev_s[i].elapsed_time(ev_e[i]) for i in range(steps)]
+    _LAST_CALL_MS[:] = times
+    kernel_ms = sum(times) / steps
     return kernel_ms, b0.elapsed_time(b1)
 
 
@@ -702,12 +722,13 @@ def run_ours(args, dist_ctx):
     def measure():
         with ClockSampler(device.index) as cs:
             k_ms, br_ms = time_device(case, args.steps, args.warmup, dist_ctx)
+            call_spread = spread(_LAST_CALL_MS)
             e_ms, h2d, d2h = time_e2e(case, args.steps, args.warmup, dist_ctx)
-        return k_ms, br_ms, e_ms, h2d, d2h, cs.summary()
+        return k_ms, br_ms, e_ms, h2d, d2h, cs.summary(), call_spread
 
-    k_ms, br_ms, e_ms, h2d, d2h, clocks = measure()
+    k_ms, br_ms, e_ms, h2d, d2h, clocks, call_spread = measure()
     if clocks_rejected(clocks):
-        k_ms, br_ms, e_ms, h2d, d2h, clocks = measure()
+        k_ms, br_ms, e_ms, h2d, d2h, clocks, call_spread = measure()
         clocks["remeasured"] = True
     k_ms, br_ms, e_ms = dist_ctx.max(k_ms), dist_ctx.max(br_ms), dist_ctx.max(e_ms)
     # a prefill workload also as 20 back-to-back calls in one CUDA graph
@@ -736,6 +757,8 @@ def run_ours(args, dist_ctx):
         "e2e": {"value": round(whole_job_value(N, work, e_ms), 3), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": roofline(w, k_ms, case.kernel, name, peaks, peak_src),
+        # this rank's per-call device times (value and ms_per_step use the mean)
+        "spread": call_spread,
         "gpu_launches": args.steps * case.launches,
         "clocks": clocks,
         "device_status": status,
@@ -758,6 +781,7 @@ def run_ours(args, dist_ctx):
         lcase = Case(leg, wl, device)
         lsteps = max(args.steps, 5)
         l_ms, _ = time_device(lcase, lsteps, max(args.warmup, 3), dist_ctx)
+        l_spread = spread(_LAST_CALL_MS)
         l_ms = dist_ctx.max(l_ms)
         hbm = bound(wl) == "hbm"
         work = algorithmic_bytes(wl) / 1e9 if hbm else algorithmic_flops(wl) / 1e12
@@ -765,6 +789,7 @@ def run_ours(args, dist_ctx):
             "workload": leg,
             "value": round(N * work / (l_ms * 1e-3), 2),
             "unit": "GB/s" if hbm else "TFLOP/s", "ms_per_step": round(l_ms, 5), "steps": lsteps,
+            "spread": l_spread,
             "gpu_launches": lsteps * lcase.launches,
             "roofline": roofline(wl, l_ms, lcase.kernel, leg, peaks, peak_src),
         }

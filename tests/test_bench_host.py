@@ -95,3 +95,10 @@ def test_profile_traffic_goes_stale_when_the_kernel_changes(tmp_path, monkeypatc
     assert bench.profiled_traffic("tcgen05", "w") == 1234.0
     (csrc / "prefill_tcgen05.cuh").write_text("kernel v2")
     assert bench.profiled_traffic("tcgen05", "w") is None
+
+
+def test_spread_of_per_call_times():
+    s = bench.spread([5, 1, 4, 2, 3, 6, 7, 8, 9, 10])
+    assert s == {"median_ms": 5.5, "p10_ms": 1, "p90_ms": 9}
+    assert bench.spread([2.0]) == {"median_ms": 2.0, "p10_ms": 2.0, "p90_ms": 2.0}
+    assert bench.spread([]) is None
