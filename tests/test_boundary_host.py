@@ -137,6 +137,12 @@ def test_plans_pick_the_intended_kernels(lib):
     for d in (64, 80, 96, 112):
         assert lib.attn_cached_plan(BF16, 1, 32, 32, 1, 2048, 2048, d, 2047) == L.KERNEL_SPLITKV
     assert lib.attn_cached_plan(BF16, 1, 32, 32, 17, 2048, 2048, 80, 2031) == L.KERNEL_TCGEN05
+    # head sizes off the tensor-core grid decode on CUDA cores; d = 256 takes
+    # the CUDA-core split-KV kernel up to 8 rows per K/V head
+    for d in (48, 72, 136, 192):
+        assert lib.attn_cached_plan(BF16, 1, 32, 32, 1, 2048, 2048, d, 2047) == L.KERNEL_SIMT
+    assert lib.attn_cached_plan(BF16, 1, 32, 32, 1, 2048, 2048, 256, 2047) == L.KERNEL_SPLITKV
+    assert lib.attn_cached_plan(BF16, 1, 32, 8, 5, 2048, 2048, 256, 2043) == L.KERNEL_SIMT
     assert lib.attn_cached_plan(F16, 32, 8, 1, 512, 4096, 4096, 128, 3584) == L.KERNEL_TCGEN05
     # head sizes the tensor-core kernel does not take fall back to CUDA cores
     assert lib.attn_prefill_plan(BF16, 1, 2, 1, 16, 40, 1) == L.KERNEL_SIMT
