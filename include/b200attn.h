@@ -29,10 +29,15 @@
  * Element type: ATTN_F32 (float), ATTN_BF16, ATTN_F16 for Q, K, V and O alike;
  * accumulation is always float32.  Output is rounded to nearest-even.
  *
- * Ownership: the caller owns every buffer.  The library allocates nothing on
- * the device, never synchronises inside a call, and enqueues its kernels on
- * `stream` (a cudaStream_t; NULL = legacy default stream).  It keeps no state
- * between calls except read-only kernel attributes.
+ * Ownership: the caller owns every buffer it passes.  No call allocates or
+ * frees device memory or synchronises (attn_device_status excepted); kernels
+ * are enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ * Two pieces of device state persist between calls, both in the library's
+ * own statically sized module memory on every device that loads it: the
+ * device status word that bounded waits and page-table checks write (read and
+ * cleared by attn_device_status), and the fixed scratch array of
+ * attn_cached_noalloc, which keeps the last such call's split partials.  The
+ * host keeps per-device kernel attributes and the scratch array's address.
  *
  * Errors: every argument is checked before anything is enqueued; on any error
  * nothing is launched and O is left untouched.  Nothing aborts the process.
@@ -128,7 +133,9 @@ ATTN_API attn_status_t attn_cached(const void* q, const void* k_hist, const void
  * whose attn_cached_workspace_size() exceeds that returns
  * ATTN_ERR_WORKSPACE and launches nothing.  The call allocates nothing: the
  * first call on each device looks up the array's device address (with that
- * device current), so make that first call before any stream capture.  All
+ * device current), so make that first call before any stream capture; the
+ * lookup is keyed on the device's context, so after a device reset the next
+ * call (again outside any capture) looks the new address up.  All
  * calls on a device share the one array and it keeps the last call's data;
  * calls that can overlap on the GPU (different streams, no ordering between
  * them) race on it and must be serialised by the caller.
@@ -216,9 +223,9 @@ ATTN_API size_t attn_cached_local_workspace_size(attn_dtype_t dtype, int64_t B, 
  * H / Hkv * Tnew <= 16, or d = 256 and H / Hkv * Tnew <= 8, run the split-KV
  * decode kernels; other
  * bf16 / fp16 shapes with d a multiple of 16 in [64, 128] (chunked prefill)
- * run the tensor-core prefill kernel, which copies whole pages: there the
- * rows of a sequence's last page past L_b are read (with zero weight) and
- * must hold finite values (zeros, or stale keys and values).  Everything
+ * run the tensor-core prefill kernel, which copies whole pages and zeroes the
+ * rows past L_b in shared memory.  Rows of a page past L_b may hold anything
+ * (NaN and inf included): no result depends on them.  Everything
  * else returns ATTN_ERR_UNSUPPORTED (float32 included).  ATTN_ERR_INVALID_ARG as for
  * attn_cached, plus: page_size not a power of two in range, max_kv_len < Tnew
  * or > max_pages * page_size, num_pages = 0, null or unaligned (4-byte) table

@@ -982,22 +982,61 @@ namespace {
 
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// The scratch array's device address, per device, with the id of the context
+// it was looked up in.
+struct NoallocAddress {
+    unsigned long long ctx_id = 0;
+    void* ptr = nullptr;
+};
+NoallocAddress g_noalloc_addr[kNoAllocMaxDevices];
+
+// Process-unique id of the current context (context ids are never reused
+// while the process lives), through the driver entry points.
+attn_status_t current_context_id(unsigned long long* id) {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 4000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+        fn = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+    });
+    if (!get_current || !get_id) return ATTN_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return ATTN_ERR_CUDA;
+    return get_id(ctx, id) == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
 
 // Device address of the scratch array on the current device.  The host-side
-// name is only a handle for the runtime; the first call on each device looks
-// the real address up (with that device current) and keeps it.
+// name is only a handle for the runtime; the address is looked up with
+// cudaGetSymbolAddress (with the device current) the first time a device is
+// used in a context and kept for that context.  A device reset ends the
+// context and reloads the module elsewhere: the next call sees a new context
+// id and looks the address up again.
 attn_status_t noalloc_scratch(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
         return ATTN_ERR_CUDA;
+    unsigned long long ctx = 0;
+    const bool have_ctx = current_context_id(&ctx) == ATTN_OK;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    NoallocAddress& a = g_noalloc_addr[dev];
+    if (!have_ctx || !a.ptr || a.ctx_id != ctx) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        // the lookup has made the device's context current if it was not yet
+        if (current_context_id(&ctx) != ATTN_OK) return ATTN_ERR_CUDA;
+        a.ptr = p;
+        a.ctx_id = ctx;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = a.ptr;
     return ATTN_OK;
 }
 
