@@ -162,3 +162,45 @@ def test_full_size_decode_sampled_rows():
         ref = oracle.paged_attention(q[b:b + 1], kp, vp, table[b:b + 1], [L],
                                      scale=1 / math.sqrt(d))
         check(got[b:b + 1], ref)
+
+
+def poison_tails(k_pages, v_pages, table, lens):
+    """Fill every page row that no sequence reads (the rows of a sequence's
+    last page past its length) with NaN, +inf and -inf in turn: a pool from
+    torch.empty or a recycled page may hold any bit pattern there."""
+    P = k_pages.shape[2]
+    bad = [float("nan"), float("inf"), float("-inf")]
+    for b, L in enumerate(lens):
+        for j in range(L, table.shape[1] * P):
+            ph, r = int(table[b, j // P]), j % P
+            k_pages[ph, :, r] = bad[j % 3]
+            v_pages[ph, :, r] = bad[(j + 1) % 3]
+
+
+NAN_TAIL_CASES = [
+    # chunked prefill on the tensor-core kernel (whole pages copied)
+    (2, 8, 1, 200, 128, [1000, 450], 64, F16),
+    (2, 16, 4, 300, 128, [777, 301], 128, BF16),
+    (1, 8, 2, 129, 64, [2001], 256, BF16),
+    (3, 8, 2, 100, 96, [100, 357, 1027], 8, BF16),
+    (2, 4, 4, 64, 80, [129, 1000], 16, F16),
+    # the split-KV decode kernels
+    (3, 8, 2, 1, 128, [1000, 37, 517], 16, BF16),
+    (2, 4, 4, 2, 256, [900, 129], 32, F16),
+]
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tnew,d,lens,page_size,dtype", NAN_TAIL_CASES)
+def test_unused_page_rows_holding_nan_or_inf_change_nothing(B, H, Hkv, Tnew, d, lens, page_size,
+                                                             dtype):
+    """Paging changes only where K/V live ("Causal Multi-Head Self-Attention",
+    Algorithm and cache boundaries): rows past a sequence's length are not part
+    of it, whatever they hold."""
+    q, kp, vp, table, kv_lens = make_paged(B, H, Hkv, Tnew, d, lens, page_size, dtype,
+                                           seed=7 + sum(lens))
+    poison_tails(kp, vp, table, lens)
+    scale = 1 / math.sqrt(d)
+    got, lse = run_gpu(q, kp, vp, table, kv_lens, scale, lse=True)
+    ref, ref_lse = oracle.paged_attention(q, kp, vp, table, lens, scale=scale, want_lse=True)
+    check(got, ref)
+    assert np.abs(lse.numpy() - ref_lse).max() <= 2e-3

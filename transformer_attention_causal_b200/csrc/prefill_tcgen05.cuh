@@ -23,6 +23,8 @@
 //   warp 1      TMEM owner (allocates all 512 columns) and single-thread MMA
 //               issuer: S_s = Q_s K_n^T (SS MMA, M=N=128), O_s += P_s V_n
 //               (TS MMA: P read straight from TMEM, N = d);
+//   warp 2      (paged caches only) zeroes the V rows of a sequence's last
+//               page past its length before P.V reads the stage;
 //   warps 4-7   softmax for slot 0, warps 8-11 softmax for slot 1: one
 //               thread per query row (TMEM lane), 128 scores in registers.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512);
@@ -259,9 +261,12 @@ __device__ __forceinline__ void prefill_unit(const PrefillParams& p, int unit, i
 }
 
 // K or V tile n of sequence b, head kvh, from a paged pool: one TMA copy per
-// page the tile spans (min(P, 128) rows each).  Rows past the sequence's end,
-// and pages whose id is out of range (reported), are read at an out-of-range
-// coordinate, which TMA fills with zeros while still counting the bytes.
+// page the tile spans (min(P, 128) rows each).  Copies that start at or past
+// the sequence's end, and pages whose id is out of range (reported), are read
+// at an out-of-range coordinate, which TMA fills with zeros while still
+// counting the bytes.  The copy that holds the sequence's last rows brings the
+// rest of its page too; those rows of a V tile are zeroed in shared memory by
+// the tail warp before P.V reads them.
 template <int DCH>
 __device__ __forceinline__ void load_kv_paged(const PrefillParams& p, uint32_t dst, const CUtensorMap* map,
                                               uint32_t bar, int n, int b, int kvh, int64_t L) {
@@ -312,7 +317,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
     uint64_t* p_ready = s_full + 2;     // [slot][half]: 4
     uint64_t* o_done = p_ready + 4;     // 2
     uint64_t* drain = o_done + 2;       // 1
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* kv_ready = drain + 1;     // NST (PAGED: V stages with their tail rows zeroed)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(kv_ready + NST);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -336,6 +342,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int i = 0; i < NST; ++i) {
             mbar_init(smem_u32(&kv_full[i]), 1);
             mbar_init(smem_u32(&kv_empty[i]), 1);
+            mbar_init(smem_u32(&kv_ready[i]), 1);
         }
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
@@ -461,7 +468,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const int64_t iV = li, iK = li + 1;
                         const int stV = int(iV % NST), stK = int(iK % NST);
                         const bool nextK = n + 1 < nmax;
-                        ok = mbar_wait(smem_u32(&kv_full[stV]), uint32_t((iV / NST) & 1), p.timeout_ns, abort_flag);
+                        ok = mbar_wait(smem_u32(PAGED ? &kv_ready[stV] : &kv_full[stV]), uint32_t((iV / NST) & 1),
+                                       p.timeout_ns, abort_flag);
                         if (ok && nextK)
                             ok = mbar_wait(smem_u32(&kv_full[stK]), uint32_t((iK / NST) & 1), p.timeout_ns,
                                            abort_flag);
@@ -512,6 +520,60 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 // every MMA issued must finish before TMEM is released
                 mma_commit(smem_u32(drain));
                 mbar_wait(smem_u32(drain), 0, p.timeout_ns, nullptr);
+            }
+        } else if (PAGED && warp == 2) {
+            // ================================================= paged V tails
+            // A copy brings whole page rows, so the rows of a sequence's last
+            // page past its length L arrive with it.  They enter P.V with
+            // weight 0, and 0 * NaN (or inf) is NaN: the result must not
+            // depend on what unused page rows hold, so they are zeroed here,
+            // in shared memory, before any MMA reads the V stage.  Every V
+            // stage passes through this warp (kv_full -> kv_ready).  K needs
+            // nothing: the scores of keys at or past L are overwritten by the
+            // mask.  Loads alternate K, V and a unit issues an even number of
+            // them, so with an even ring every use of a V stage is a V load
+            // and kv_ready's phases follow kv_full's.
+            static_assert(NST % 2 == 0, "V loads must keep to their own stages");
+            const int64_t copy_rows = min(int64_t(1) << p.page_shift, int64_t(128));
+            int64_t li = 0;
+            bool ok = true;
+            for (int pass = 0; ok; ++pass) {
+                const int unit = prefill_pass_unit(pass);
+                if (unit >= n_units) break;
+                int b, kvh;
+                SlotInfo slot[2];
+                prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                const int nmax = max(slot[0].n_kv, slot[1].n_kv);
+                const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
+                                 : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
+                const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * (nmax - nmin);
+                const int64_t L = slot[0].S;
+                // rows [L, end of the copy holding row L - 1) came from the pool
+                const int64_t tail_end = (L + copy_rows - 1) / copy_rows * copy_rows;
+                for (int i = 0; i < n_loads && ok; ++i, ++li) {
+                    if ((i & 1) == 0) continue;
+                    const int st = int(li % NST);
+                    ok = mbar_wait(smem_u32(&kv_full[st]), uint32_t((li / NST) & 1), p.timeout_ns, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    const int64_t t0 = int64_t(nmin + (i >> 1)) * 128;
+                    const int r0 = int(max64(0, min64(128, L - t0)));
+                    const int r1 = int(max64(0, min64(128, tail_end - t0)));
+                    if (r1 > r0) {
+                        // whole 128-byte rows: the swizzle only permutes 16-byte
+                        // pieces within a row
+                        const uint32_t dst = sRing + uint32_t(st * DCH) * kChunkBytes + uint32_t(r0) * 128u;
+                        const int per_chunk = (r1 - r0) * 8;
+                        for (int x = lane; x < DCH * per_chunk; x += 32) {
+                            const int c = x / per_chunk;
+                            const uint32_t a = dst + uint32_t(c) * kChunkBytes + uint32_t(x - c * per_chunk) * 16u;
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&kv_ready[st]));
+                }
             }
         }
     } else {
