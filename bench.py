@@ -5,13 +5,15 @@
 
 One step = one call of the library on one batch of the workload (default: the
 BitNet-3B-shaped causal MHA prefill, B=1, H=32, T=2048, d=80, bf16).  The
-line also carries the cached-decode half of the metric (GQA decode, B=64,
+line also carries the GQA prefill (B=8, H=16/8, T=4096, d=128, bf16), the MQA
+chunked prefill against a cache (B=32, H=8/1, 512 new tokens at 3584 over 4096
+keys, d=128, fp16), the cached-decode half of the metric (GQA decode, B=64,
 H=32/8, S=8192, d=128, bf16), the same decode over a paged cache (64-token
 pages), the GQA prefill with a 2048-key local window (B=2, T=8192), the
 KV-cache append with RoPE on K of the GQA prefill's keys and values (B=8,
 Hkv=8, 4096 tokens, d=128, bf16), and the backward pass of the GQA prefill
 (dQ, dK, dV from the forward's O and row statistic), each measured the same
-way with its own roofline.
+way with its own roofline and its own bounded oracle baseline.
 
 Timing: W untimed steps, then exactly K timed steps bracketed by a barrier and
 torch.cuda.synchronize() on both sides.  Before every timed call L2 is flushed
@@ -70,6 +72,10 @@ WORKLOADS = {
                                         Tnew=4096, start=0, S=4096, d=128, base=10000.0),
 }
 DEFAULT_WORKLOAD = "bitnet3b_mha_prefill_bf16"
+GQA_PREFILL_WORKLOAD = "gqa16x8_prefill_bf16"
+MQA_CHUNKED_WORKLOAD = "mqa_chunked_prefill_f16"
+# seconds of oracle work behind each leg's cpu_baseline (the line's own: 10 s)
+LEG_BASELINE_S = 3.0
 DECODE_WORKLOAD = "gqa_decode_bf16"
 APPEND_WORKLOAD = "kv_append_rope_gqa16x8_bf16"
 WINDOW_WORKLOAD = "gqa_prefill_swa_bf16"
@@ -262,19 +268,35 @@ def kernel_source_sha(kernel: str) -> str:
         return hashlib.sha256(fh.read()).hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this kernel and
-    workload, or None when there is none or the kernel changed since."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+PROFILED_KEYS = ("dram_bytes_per_launch", "tensor_pipe_active_pct", "dram_throughput_pct")
+
+
+def profiled(kernel: str, workload: str):
+    """Figures of the committed ncu summary of this kernel and workload
+    (profiles/<kernel>_<workload>.md): DRAM bytes per launch and, where
+    captured, the tensor-pipe active and DRAM throughput percentages.  Empty
+    when there is no summary or the kernel source changed since it was taken."""
+    rel = os.path.join("profiles", f"{kernel}_{workload}.md")
     try:
-        text = open(path).read()
+        text = open(os.path.join(ROOT, rel)).read()
     except OSError:
-        return None
-    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        return {}
     m_sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    if not m_bytes or not m_sha or m_sha.group(1) != kernel_source_sha(kernel):
-        return None
-    return float(m_bytes.group(1))
+    if not m_sha or m_sha.group(1) != kernel_source_sha(kernel):
+        return {}
+    out = {}
+    for key in PROFILED_KEYS:
+        m = re.search(key + r":\s*([0-9.eE+]+)", text)
+        if m:
+            out[key] = float(m.group(1))
+    if out:
+        out["source"] = rel
+    return out
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None."""
+    return profiled(kernel, workload).get("dram_bytes_per_launch")
 
 
 # ------------------------------------------------------------------ our implementation
@@ -561,10 +583,16 @@ def roofline(w, kernel_ms, kernel, name, peaks, peak_src):
         # a kernel timed alone: the burst GEMM figure
         peak = peaks["bf16_tflops"]
         unit = "TFLOP/s"
-    return {"bound": bound(w), "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+    prof = profiled(kernel, name)
+    line = {"bound": bound(w), "achieved": round(achieved, 2), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
-            if peak_src == "measured" else "fallback", "traffic": profiled_traffic(kernel, name),
-            "kernel": kernel}
+            if peak_src == "measured" else "fallback",
+            "traffic": prof.get("dram_bytes_per_launch"), "kernel": kernel}
+    if prof:
+        # from the committed ncu summary (same kernel source): percentages of
+        # the capture's elapsed cycles / of peak DRAM throughput
+        line["ncu"] = {k: v for k, v in prof.items() if k != "dram_bytes_per_launch"}
+    return line
 
 
 class OracleSample:
@@ -769,9 +797,12 @@ def run_ours(args, dist_ctx):
                          "value": round(whole_job_value(N, gwork, g_ms), 3), "unit": "TFLOP/s",
                          "note": "20 calls captured in one CUDA graph, L2 flushed before each replay; "
                                  "not counted in gpu_launches"}
-    legs = [] if args.no_decode else [("decode", DECODE_WORKLOAD), ("paged", PAGED_WORKLOAD),
+    legs = [] if args.no_decode else [("gqa_prefill", GQA_PREFILL_WORKLOAD),
+                                      ("mqa_chunked_prefill", MQA_CHUNKED_WORKLOAD),
+                                      ("decode", DECODE_WORKLOAD), ("paged", PAGED_WORKLOAD),
                                       ("window", WINDOW_WORKLOAD), ("append", APPEND_WORKLOAD),
                                       ("backward", BACKWARD_WORKLOAD)]
+    baselines = dist_ctx.rank == 0 and N == 1 and not args.no_cpu_baseline
     del case
     for key, leg in legs:
         if leg == name:
@@ -794,7 +825,9 @@ def run_ours(args, dist_ctx):
             "roofline": roofline(wl, l_ms, lcase.kernel, leg, peaks, peak_src),
         }
         del lcase
-    if dist_ctx.rank == 0 and N == 1 and not args.no_cpu_baseline:
+        if baselines:
+            line[key]["cpu_baseline"] = cpu_baseline(wl, leg, target_s=LEG_BASELINE_S)
+    if baselines:
         line["cpu_baseline"] = cpu_baseline(w, name)
     if dist_ctx.rank == 0:
         print(json.dumps(line), flush=True)
