@@ -39,10 +39,14 @@ def test_bounded_waits_report_a_timeout_and_leave_the_context_usable():
     assert attn.cached_plan(torch.bfloat16, 2, 8, 2, 1, 1000, 1000, 128, 999) == "splitkv"
     pq, pk, pv, dq, dk, dv = (t.cuda() for t in (pq, pk, pv, dq, dk, dv))
     assert attn.device_status(reset=True) == _lib.OK
+    # a head size of 80 (the second 64-column chunk partly filled) too
+    sq, sk, sv = (t.cuda() for t in inputs.qkv(1, 3, 3, 300, 300, 80, torch.bfloat16, seed=33))
     try:
         attn.set_wait_timeout_ns(20_000_000)  # 20 ms
         lib.attn_test_set_flags(1)
         attn.prefill(pq, pk, pv, scale=scale)
+        assert attn.device_status(reset=True) == _lib.ERR_DEVICE_TIMEOUT
+        attn.prefill(sq, sk, sv, scale=1 / math.sqrt(80))
         assert attn.device_status(reset=True) == _lib.ERR_DEVICE_TIMEOUT
         attn.cached(dq, dk, dv, start_pos=999, scale=scale)
         assert attn.device_status(reset=True) == _lib.ERR_DEVICE_TIMEOUT
@@ -56,6 +60,10 @@ def test_bounded_waits_report_a_timeout_and_leave_the_context_usable():
     assert err.max() <= 1.5e-2 and err.mean() <= 2e-3
     out = attn.cached(dq, dk, dv, start_pos=999, scale=scale).float().cpu().numpy()
     ref = oracle(dq.cpu(), dk.cpu(), dv.cpu(), scale=scale, causal=True, start_pos=999)
+    err = np.abs(out - ref)
+    assert err.max() <= 1.5e-2 and err.mean() <= 2e-3
+    out = attn.prefill(sq, sk, sv, scale=1 / math.sqrt(80)).float().cpu().numpy()
+    ref = oracle(sq.cpu(), sk.cpu(), sv.cpu(), scale=1 / math.sqrt(80), causal=True)
     err = np.abs(out - ref)
     assert err.max() <= 1.5e-2 and err.mean() <= 2e-3
     assert attn.device_status() == _lib.OK
