@@ -278,6 +278,25 @@ attn_status_t run_simt(const Problem& pb, const void* q, const void* k, const vo
     return launch_status();
 }
 
+// The split merge, launched as a programmatic dependent of the decode kernel
+// just enqueued on `stream`: its launch overlaps the decode's tail and it
+// waits (griddepcontrol.wait) for the decode grid's results.
+template <typename T, int D>
+attn_status_t launch_combine(const DecodeParams& dp, cudaStream_t stream) {
+    const int64_t rows = int64_t(dp.B) * dp.Hkv * dp.Rv;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(unsigned((rows + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<T, D>, dp) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 template <typename T, int D, int R, int MODE>
 attn_status_t launch_decode_RP(const DecodeParams& dp, cudaStream_t stream) {
     constexpr size_t smem = DecodeShape<D, R>::smem_bytes(sizeof(T));
@@ -286,11 +305,7 @@ attn_status_t launch_decode_RP(const DecodeParams& dp, cudaStream_t stream) {
     dim3 grid(unsigned(dp.nsplit), unsigned(dp.B * dp.Hkv));
     kern<<<grid, 160, smem, stream>>>(dp);
     if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
-    if (dp.nsplit > 1) {
-        const int64_t rows = int64_t(dp.B) * dp.Hkv * dp.Rv;
-        decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, stream>>>(dp);
-        return launch_status();
-    }
+    if (dp.nsplit > 1) return launch_combine<T, D>(dp, stream);
     return ATTN_OK;
 }
 
@@ -320,11 +335,7 @@ attn_status_t launch_decode_mma_k(const CUtensorMap& mk, const CUtensorMap& mv, 
     dim3 grid(unsigned(dp.nsplit), unsigned(dp.B * dp.Hkv));
     kern<<<grid, kDecMmaThreads, smem, stream>>>(mk, mv, dp);
     if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
-    if (dp.nsplit > 1) {
-        const int64_t rows = int64_t(dp.B) * dp.Hkv * dp.Rv;
-        decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, stream>>>(dp);
-        return launch_status();
-    }
+    if (dp.nsplit > 1) return launch_combine<T, D>(dp, stream);
     return ATTN_OK;
 }
 

@@ -90,6 +90,9 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         fence_mbar_init();
     }
     __syncthreads();
+    // the split merge (a programmatic dependent) may be launched now; it
+    // waits for this grid to finish before it reads anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == NW) {
         // ============================================ TMA producer (lane 0)

@@ -226,6 +226,8 @@ decode_splitkv_kernel(const DecodeParams p) {
         fence_mbar_init();
     }
     __syncthreads();
+    // the split merge (a programmatic dependent) may be launched now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const T* kg = static_cast<const T*>(p.k) + (size_t(unit) * p.S_cap) * D;
     const T* vg = static_cast<const T*>(p.v) + (size_t(unit) * p.S_cap) * D;
@@ -528,6 +530,10 @@ decode_splitkv_kernel(const DecodeParams p) {
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
 decode_combine_kernel(const DecodeParams p) {
+    // launched as a programmatic dependent of the decode kernel: its launch
+    // overlaps the decode's tail, and this wait holds it until the decode
+    // grid has finished and its partials are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row = int64_t(blockIdx.x) * 4 + warp;  // over units * Rv
     const int64_t nrows = int64_t(p.B) * p.Hkv * p.Rv;
