@@ -162,3 +162,40 @@ def test_full_size_group_of_the_benchmark_workload():
         check("dq", dq[b:b + 1, hs], ref[0], BF16)
         check("dk", dk[b:b + 1, kvh:kvh + 1], ref[1], BF16)
         check("dv", dv[b:b + 1, kvh:kvh + 1], ref[2], BF16)
+
+
+def test_full_size_backward_sampled_heads_and_sums():
+    """The backward workload at full size (B=8, 16 query / 8 K/V heads,
+    T=4096, d=128, bf16), whose key and query tiles are worked through in
+    several groups of heads: dQ of three (b, h) slices and dK, dV of one
+    (b, K/V head) against the oracle on those heads alone (a head's dQ needs
+    only its own rows; a K/V head's dK and dV only its G query heads), and for
+    every (b, K/V head) the sums that hold at any size: sum_j dV_j = sum of
+    dO over its query heads (each probability row sums to 1) and
+    sum_j dK_j = 0 (shifting every key leaves each softmax row unchanged)."""
+    B, H, Hkv, T, d = 8, 16, 8, 4096, 128
+    G = H // Hkv
+    q, k, v = inputs.qkv(B, H, Hkv, T, T, d, BF16, seed=9)
+    dout = inputs.upstream(B, H, T, d, BF16, seed=9)
+    scale = 1 / math.sqrt(d)
+    dq, dk, dv = run_gpu(q, k, v, dout, scale, True)
+    u = UNIT[BF16]
+    for b, h in ((0, 0), (3, 9), (7, 15)):
+        kvh = h // G
+        ref, _, _ = oracle.attention_backward(q[b:b + 1, h:h + 1], k[b:b + 1, kvh:kvh + 1],
+                                              v[b:b + 1, kvh:kvh + 1], dout[b:b + 1, h:h + 1],
+                                              scale=scale, causal=True)
+        check(f"dq[{b},{h}]", dq[b:b + 1, h:h + 1], ref, BF16)
+    b, kvh = 5, 6
+    _, ref_dk, ref_dv = oracle.attention_backward(q[b:b + 1, kvh * G:(kvh + 1) * G],
+                                                  k[b:b + 1, kvh:kvh + 1], v[b:b + 1, kvh:kvh + 1],
+                                                  dout[b:b + 1, kvh * G:(kvh + 1) * G],
+                                                  scale=scale, causal=True)
+    check("dk[5,6]", dk[b:b + 1, kvh:kvh + 1], ref_dk, BF16)
+    check("dv[5,6]", dv[b:b + 1, kvh:kvh + 1], ref_dv, BF16)
+    dv64, dk64 = dv.double(), dk.double()
+    do_sum = dout.double().reshape(B, Hkv, G, T, d).sum(dim=(2, 3))        # [B, Hkv, d]
+    dv_sum = dv64.sum(dim=2)
+    assert torch.all((dv_sum - do_sum).abs() <= 8 * u * do_sum.abs().amax(dim=-1, keepdim=True) + 1e-2)
+    dk_scale = dk64.abs().sum(dim=2)
+    assert torch.all(dk64.sum(dim=2).abs() <= 8 * u * dk_scale + 1e-3)

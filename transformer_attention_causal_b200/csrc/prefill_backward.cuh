@@ -68,6 +68,7 @@ struct BwdParams {
     int B, H, Hkv, G, T, Tpad, d, causal;
     int window;           // local window w (causal): row i reads keys i - w < j <= i; 0: none
     int n_t;              // ceil(T / 128)
+    int group_kv, group_q; // work order (grouped_order): items per L2 group, dK/dV and dQ kernels
     float scale, scale_log2;
     uint64_t timeout_ns;
     uint32_t test_flags;  // kTestSkipLoads: issue no copies (timeout-path tests)
@@ -231,8 +232,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bk = int(blockIdx.x % unsigned(p.B * p.Hkv));
-    const int kt = int(blockIdx.x / unsigned(p.B * p.Hkv));   // heaviest (kt = 0) first
+    // (b, K/V head) in groups whose Q and dO tiles fit in L2 together, each
+    // group heaviest (kt = 0) first
+    int kt, bk;
+    grouped_order(blockIdx.x, p.B * p.Hkv, p.n_t, p.group_kv, kt, bk);
     const int b = bk / p.Hkv, kvh = bk % p.Hkv;
     const int q_lo = p.causal ? kt : 0;
     // with a window only the query tiles whose rows reach this key tile
@@ -495,8 +498,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = int(blockIdx.x % unsigned(p.B * p.H));
-    const int qt = p.n_t - 1 - int(blockIdx.x / unsigned(p.B * p.H));   // heaviest first
+    // (b, head) in groups whose K and V tiles fit in L2 together, each group
+    // heaviest (last query tile) first
+    int lvl, bh;
+    grouped_order(blockIdx.x, p.B * p.H, p.n_t, p.group_q, lvl, bh);
+    const int qt = p.n_t - 1 - lvl;
     const int b = bh / p.H, h = bh % p.H;
     const int bk = b * p.Hkv + h / p.G;
     // key tiles n_first .. n_first + n_kv - 1 (with a window: from the first

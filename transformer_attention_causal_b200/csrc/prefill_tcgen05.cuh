@@ -58,6 +58,7 @@ struct PrefillParams {
     int n_qb;            // ceil(Tq / 128)
     int units_per_level;
     int n_levels;        // units = units_per_level * n_levels, heaviest level first
+    int group;           // units of a level taken together (grouped_order)
     float scale_log2;    // |scale| * log2(e) (1 when scale = 0)
     int score_mode;      // 0: scale > 0; 1: scale < 0 (scores negated); 2: scale = 0 (scores zeroed)
     uint64_t timeout_ns;
@@ -221,13 +222,37 @@ __device__ __forceinline__ void issue_PV(uint64_t dV0, uint32_t tmem, uint32_t i
                (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// Work order with L2 locality.  The units are `per_level` items (batch
+// entries and heads) times `n_levels` levels of decreasing work.  Walking
+// level by level puts one tile of every item in flight at once, and at
+// several GB of K/V the tiles a CTA reuses are gone from L2 by then; so the
+// items are taken in groups of `group` consecutive ones whose tiles fit in L2
+// together, each group heaviest level first.  Unit -> (level, item).
+__host__ __device__ __forceinline__ void grouped_order(int unit, int per_level, int n_levels, int group,
+                                                       int& level, int& item) {
+    // 32-bit throughout: the planners keep every unit count below 2^31
+    const int full = per_level / group;             // whole groups
+    const int span = group * n_levels;
+    if (unit < full * span) {
+        const int g = unit / span, r = unit % span;
+        level = r / group;
+        item = g * group + r % group;
+    } else {
+        const int last = per_level - full * group;  // > 0 here
+        const int r = unit - full * span;
+        level = r / last;
+        item = full * group + r % last;
+    }
+}
+
 // The unit of work a CTA does at pass `unit`: its batch entry, K/V head and
-// two slots (heaviest first: the longest causal row range first).
+// two slots (heaviest first within a group of K/V heads: the longest causal
+// row range first).
 template <bool WINDOW, bool PAGED>
 __device__ __forceinline__ void prefill_unit(const PrefillParams& p, int unit, int& b, int& kvh,
                                              SlotInfo (&slot)[2]) {
-    const int level = unit / p.units_per_level;
-    const int rem = unit % p.units_per_level;
+    int level, rem;
+    grouped_order(unit, p.units_per_level, p.n_levels, p.group, level, rem);
     int h0, h1, qb0, qb1;
     if (p.pair_mode == 0) {
         const int half = p.G / 2;
