@@ -294,10 +294,6 @@ def profiled(kernel: str, workload: str):
     return out
 
 
-def profiled_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, or None."""
-    return profiled(kernel, workload).get("dram_bytes_per_launch")
-
 
 # ------------------------------------------------------------------ our implementation
 

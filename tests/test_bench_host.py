@@ -91,10 +91,19 @@ def test_profile_traffic_goes_stale_when_the_kernel_changes(tmp_path, monkeypatc
     (tmp_path / "profiles").mkdir()
     sha = bench.kernel_source_sha("tcgen05")
     prof = tmp_path / "profiles" / "tcgen05_w.md"
-    prof.write_text(f"dram_bytes_per_launch: 1234\nkernel_source_sha256_16: {sha}\n")
-    assert bench.profiled_traffic("tcgen05", "w") == 1234.0
+    prof.write_text(f"dram_bytes_per_launch: 1234\ntensor_pipe_active_pct: 45.5\n"
+                    f"kernel_source_sha256_16: {sha}\n")
+    got = bench.profiled("tcgen05", "w")
+    assert got["dram_bytes_per_launch"] == 1234.0 and got["tensor_pipe_active_pct"] == 45.5
+    assert got["source"] == "profiles/tcgen05_w.md" and "dram_throughput_pct" not in got
+    w = {"kind": "prefill", "dtype": "bf16", "B": 1, "H": 2, "Hkv": 1, "T": 256, "d": 64}
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    line = bench.roofline(w, 1.0, "tcgen05", "w", peaks, "measured")
+    assert line["traffic"] == 1234.0 and line["ncu"]["tensor_pipe_active_pct"] == 45.5
     (csrc / "prefill_tcgen05.cuh").write_text("kernel v2")
-    assert bench.profiled_traffic("tcgen05", "w") is None
+    assert bench.profiled("tcgen05", "w") == {}
+    line = bench.roofline(w, 1.0, "tcgen05", "w", peaks, "measured")
+    assert line["traffic"] is None and "ncu" not in line
 
 
 def test_spread_of_per_call_times():
