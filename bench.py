@@ -365,9 +365,11 @@ class Case:
             need = attn.cached_workspace_size(dt, w["B"], w["H"], w["Hkv"], Tq, S, w["d"],
                                               w["start"])
             self.ws = torch.empty(need, dtype=torch.uint8, device=device) if need else None
-        # launches of this library's kernels per call
+        # launches of this library's kernels per call: a workspace means a
+        # second kernel merges partial results (the split-KV decode's splits,
+        # or the pieces of a chunked prefill's last pass of units)
         self.launches = 1
-        if self.kernel == "splitkv" and self.ws is not None:
+        if self.kernel in ("splitkv", "tcgen05") and self.ws is not None:
             self.launches = 2
 
     def call(self, bufs=None, stream=None):

@@ -112,7 +112,11 @@ ATTN_API attn_status_t attn_prefill(const void* q, const void* k, const void* v,
  *   o [B,H,Tnew,d]; lse nullable [B,H,Tnew].  Always causal.
  *   workspace: device buffer of at least attn_cached_workspace_size() bytes,
  *   16-byte aligned (may be NULL when that size is 0); its contents on entry
- *   do not matter and are clobbered.
+ *   do not matter and are clobbered.  It holds fp32 partial results: the
+ *   split-KV decode's per-split rows, or, for a chunked prefill on the
+ *   tensor-core kernel whose last pass of work units would leave most SMs
+ *   idle, those units' rows computed in 2-4 pieces of the key range (merged
+ *   by a second kernel on the same stream).
  */
 ATTN_API attn_status_t attn_cached(const void* q, const void* k_hist, const void* v_hist, void* o,
                           float* lse, attn_dtype_t dtype, int64_t B, int64_t H, int64_t Hkv,
@@ -127,10 +131,11 @@ ATTN_API attn_status_t attn_cached(const void* q, const void* k_hist, const void
  * pages have no counterpart to this call; it exists for such callers only.
  *
  * Same operation, arguments, layouts and errors as attn_cached minus
- * `workspace` / `workspace_bytes`.  The split-KV partials go to one
- * library-owned device array of ATTN_NOALLOC_SCRATCH_BYTES (16 MiB), present
- * on every GPU that loads the library until the process exits.  A problem
- * whose attn_cached_workspace_size() exceeds that returns
+ * `workspace` / `workspace_bytes`.  The partials go to one library-owned
+ * device array of ATTN_NOALLOC_SCRATCH_BYTES (16 MiB), present on every GPU
+ * that loads the library until the process exits.  A chunked prefill cuts
+ * fewer pieces (or none) rather than need more than the array; a split-KV
+ * decode whose attn_cached_workspace_size() exceeds it returns
  * ATTN_ERR_WORKSPACE and launches nothing.  The call allocates nothing: the
  * first call on each device looks up the array's device address (with that
  * device current), so make that first call before any stream capture; the
@@ -216,7 +221,7 @@ ATTN_API size_t attn_cached_local_workspace_size(attn_dtype_t dtype, int64_t B, 
  *     max_pages * page_size.
  *   page_size: a power of two, 8 .. 2^20.
  *   workspace: at least attn_cached_paged_workspace_size() bytes, 16-byte
- *     aligned; may be NULL when that size is 0.
+ *     aligned; may be NULL when that size is 0 (partials as for attn_cached).
  * The device arrays are read, never written; entries out of range are
  * reported through attn_device_status() as ATTN_ERR_DEVICE_INDEX.
  * Kernels: bf16 / fp16 with d a multiple of 16 in [64, 128] and

@@ -151,6 +151,27 @@ def test_plans_pick_the_intended_kernels(lib):
     assert lib.attn_prefill_plan(BF16, 1, 3, 2, 16, 64, 1) == -1
 
 
+def test_chunked_prefill_tail_pieces_workspace(lib):
+    """The tensor-core chunked prefill cuts the units of its last pass into
+    pieces of their key range when that pass would leave most of the 148 SMs
+    idle; the workspace holds each piece's fp32 O rows and one log2-sum-exp
+    per row."""
+    F16 = 2
+    # MQA chunked prefill (B=32, H=8/1, 512 new tokens at 3584 over 4096
+    # keys, d=128): 512 units, 3 full passes, 68 units left, 2 pieces each
+    assert lib.attn_cached_workspace_size(F16, 32, 8, 1, 512, 4096, 128, 3584) == 68 * 2 * 2 * 128 * 129 * 4
+    # a single unit (B=1, H=2/1, 64 new tokens over 4064 keys, d=112): 4 pieces
+    assert lib.attn_cached_workspace_size(BF16, 1, 2, 1, 64, 4064, 112, 4000) == 4 * 2 * 128 * 113 * 4
+    # 2048 units (13 full passes, 124 left of 148): not cut
+    assert lib.attn_cached_workspace_size(BF16, 8, 16, 8, 4096, 4096, 128, 0) == 0
+    # a short history: no piece would keep 4 key tiles
+    assert lib.attn_cached_workspace_size(F16, 2, 8, 1, 200, 500, 128, 300) == 0
+    # a local window is never cut
+    assert lib.attn_cached_local_workspace_size(F16, 32, 8, 1, 512, 4096, 128, 3584, 1024) == 0
+    # the paged form plans with the length bound
+    assert lib.attn_cached_paged_workspace_size(F16, 32, 8, 1, 512, 128, 4096) == 68 * 2 * 2 * 128 * 129 * 4
+
+
 def test_workspace_size_is_zero_without_splits(lib):
     # a single long sequence on one K/V head still splits; a tiny history does not
     assert lib.attn_cached_workspace_size(BF16, 1, 4, 4, 1, 64, 128, 63) == 0

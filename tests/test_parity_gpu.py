@@ -159,6 +159,12 @@ CACHED_CASES = [
     (F16, 2, 8, 1, 200, 300, 500, 520, 128, "tcgen05"),     # MQA chunked prefill
     (BF16, 1, 4, 2, 64, 37, 101, 101, 80, "tcgen05"),       # unaligned start
     (BF16, 1, 2, 2, 100, 400, 600, 640, 64, "tcgen05"),     # history past the last query
+    # chunked prefills whose units are fewer than half the SMs: each unit is
+    # cut into pieces of its key range, merged by a second kernel
+    (F16, 2, 8, 1, 256, 1792, 2048, 2048, 128, "tcgen05"),   # 16 units, 3 pieces each
+    (BF16, 1, 4, 4, 300, 1100, 1400, 1400, 80, "tcgen05"),   # MHA, an empty second slot, 2 pieces
+    (BF16, 1, 8, 2, 130, 1000, 1130, 1152, 64, "tcgen05"),   # d = 64, unaligned start, 2 pieces
+    (BF16, 1, 2, 1, 64, 4000, 4064, 4096, 112, "tcgen05"),   # one unit in 4 pieces
     (F32, 2, 4, 2, 5, 60, 70, 72, 32, "simt"),
     (BF16, 1, 4, 2, 3, 20, 30, 30, 40, "simt"),
 ]

@@ -91,3 +91,39 @@ def test_noalloc_matches_cached_on_two_calls_in_a_row():
         err = np.abs(got - exact)
         assert err.max() <= 1.5e-2 and err.mean() <= 2e-3, (seed, err.max(), err.mean())
     assert attn.device_status() == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_chunked_prefill_pieces_match_the_oracle():
+    """A chunked prefill whose 16 units are cut into pieces of their key range:
+    the pieces' partials go to the fixed array too.  Two calls in a row, each
+    against the fp64 oracle on every row."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import transformer_attention_causal_b200 as attn
+    from oracle import attention as oracle_attention
+    from transformer_attention_causal_b200.build import build
+
+    build()
+    lib, fn = noalloc_fn()
+    B, H, Hkv, Tnew, S, d = 2, 8, 1, 256, 2048, 128
+    start = S - Tnew
+    scale = 1.0 / math.sqrt(d)
+    need = lib.attn_cached_workspace_size(BF16, B, H, Hkv, Tnew, S, d, start)
+    assert 0 < need <= SCRATCH_BYTES  # pieces, and they fit the array
+    stream = torch.cuda.current_stream()
+    for seed in (31, 32):
+        q, k, v = inputs.qkv(B, H, Hkv, Tnew, S, d, torch.bfloat16, seed=seed)
+        qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+        out = torch.full_like(qd, float("nan"))
+        rc = fn(ctypes.c_void_p(qd.data_ptr()), ctypes.c_void_p(kd.data_ptr()),
+                ctypes.c_void_p(vd.data_ptr()), ctypes.c_void_p(out.data_ptr()), None, BF16, B, H,
+                Hkv, Tnew, S, S, d, start, scale, ctypes.c_void_p(stream.cuda_stream))
+        assert rc == _lib.OK, _lib.status_string(rc)
+        torch.cuda.synchronize()
+        got = out.double().cpu().numpy()
+        exact = oracle_attention(q, k, v, scale=scale, causal=True, start_pos=start)
+        err = np.abs(got - exact)
+        assert np.all(np.isfinite(err))
+        assert err.max() <= 1.5e-2 and err.mean() <= 2e-3, (seed, err.max(), err.mean())
+    assert attn.device_status() == 0

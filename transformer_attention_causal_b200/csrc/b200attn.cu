@@ -54,6 +54,7 @@ struct Plan {
     size_t ws_bytes = 0;
     // tcgen05 prefill
     int dch = 0, pair_mode = 0, n_qb = 0, units_per_level = 0, n_levels = 0, group = 1;
+    int n_whole = 0, split = 1;   // units done whole; pieces per later unit
 };
 
 bool empty_problem(const Problem& pb) { return pb.B == 0 || pb.H == 0 || pb.Tq == 0; }
@@ -145,7 +146,42 @@ int l2_group(int64_t run_bytes, int64_t per_run, int64_t per_level) {
     return int(std::max<int64_t>(1, std::min<int64_t>(runs * std::max<int64_t>(per_run, 1), per_level)));
 }
 
-void plan_prefill_tc(const Problem& pb, Plan& pl) {
+// Key tiles of the first query tile's slot (the lightest units' range).
+int64_t first_tile_keys(const Problem& pb) {
+    const int64_t end = pb.causal ? std::min(pb.S, pb.start_pos + std::min<int64_t>(128, pb.Tq)) : pb.S;
+    return (end + 127) / 128;
+}
+
+// Tail split of the tensor-core prefill (cached calls, no window): with U
+// units on g CTAs (one per SM), the last pass holds R = U mod g units (all of
+// them when U < g).  When R is at most half the CTAs, those units are cut into
+// `split` pieces of at least 4 key tiles each (at most kMergeMaxSplit,
+// R * split <= g), so the last pass costs about 1 / split of a unit instead of
+// a whole one while the other CTAs would idle.  Only calls of at most 8 full passes, where that tail is worth the
+// pieces' fp32 partials and the merge launch.  The pieces' workspace must fit
+// `ws_cap` (fewer pieces otherwise).
+void plan_tail_split(const Problem& pb, Plan& pl, size_t ws_cap) {
+    pl.n_whole = pl.units_per_level * pl.n_levels;
+    pl.split = 1;
+    if (!pb.cached || pb.window > 0) return;
+    const int64_t U = int64_t(pl.units_per_level) * pl.n_levels;
+    const int64_t g = kPlanSMs;
+    const int64_t full = U / g, R = U % g;
+    if (R == 0 || 2 * R > g || full > 8) return;
+    int64_t split = std::min<int64_t>(std::min<int64_t>(g / R, kMergeMaxSplit), first_tile_keys(pb) / 4);
+    for (; split >= 2; --split) {
+        const size_t bytes = size_t(R * split) * 2 * 128 * size_t(pb.d + 1) * sizeof(float);
+        const size_t ws = (bytes + 255) & ~size_t(255);
+        if (ws <= ws_cap) {
+            pl.n_whole = int(full * g);
+            pl.split = int(split);
+            pl.ws_bytes = ws;
+            return;
+        }
+    }
+}
+
+void plan_prefill_tc(const Problem& pb, Plan& pl, size_t ws_cap) {
     pl.kernel = ATTN_KERNEL_TCGEN05;
     const int64_t G = pb.H / pb.Hkv;
     pl.dch = pb.d <= 64 ? 1 : 2;
@@ -164,9 +200,12 @@ void plan_prefill_tc(const Problem& pb, Plan& pl) {
     // then reads the same few K/V heads; DRAM was only ~30 % busy), so the
     // forward keeps the heaviest-first order across all items.
     pl.group = pl.units_per_level;
+    plan_tail_split(pb, pl, ws_cap);
 }
 
-attn_status_t make_plan(const Problem& pb, Plan& pl) {
+// `ws_cap`: the most workspace the call can be given (the no-allocation
+// entry point's fixed array); plans that would need more use less.
+attn_status_t make_plan(const Problem& pb, Plan& pl, size_t ws_cap = SIZE_MAX) {
     attn_status_t st = check_shape(pb);
     if (st != ATTN_OK) return st;
     pl = Plan();
@@ -184,7 +223,7 @@ attn_status_t make_plan(const Problem& pb, Plan& pl) {
     if (pb.d % 16 == 0 && pb.d >= 64 && pb.d <= 128 &&
         (pb.B * pb.Hkv * std::max<int64_t>(G / 2, 1) * ((pb.Tq + 127) / 128)) < (int64_t(1) << 31) &&
         pb.S_cap * pb.d * 2 < (int64_t(1) << 40)) {
-        plan_prefill_tc(pb, pl);
+        plan_prefill_tc(pb, pl, ws_cap);
         return ATTN_OK;
     }
     pl.kernel = ATTN_KERNEL_SIMT;
@@ -446,12 +485,39 @@ attn_status_t launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk
         st != ATTN_OK)
         return st;
     kern<<<unsigned(grid), kPfThreads, smem, stream>>>(mq, mk, mv, pp);
-    return launch_status();
+    if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
+    if (pp.split <= 1) return ATTN_OK;
+    // the pieces' merge, as a programmatic dependent (as the decode's combine)
+    const int64_t rows = int64_t(pp.units_per_level * pp.n_levels - pp.n_whole) * 256;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(unsigned((rows + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_merge_kernel<T>, pp) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Work items of a plan and the pieces' workspace.
+void set_items(PrefillParams& pp, const Plan& pl, const Problem& pb, void* ws) {
+    pp.n_whole = pl.n_whole;
+    pp.split = pl.split;
+    pp.ws_o = nullptr;
+    pp.ws_lse = nullptr;
+    if (pl.split > 1) {
+        const size_t rows = size_t(pl.units_per_level * pl.n_levels - pl.n_whole) * pl.split * 256;
+        pp.ws_o = static_cast<float*>(ws);
+        pp.ws_lse = pp.ws_o + rows * size_t(pb.d);
+    }
 }
 
 template <typename T, int DCH>
 attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q, const void* k,
-                                const void* v, void* o, float* lse, float scale,
+                                const void* v, void* o, float* lse, float scale, void* ws,
                                 cudaStream_t stream) {
     if (get_encoder() != ATTN_OK) return ATTN_ERR_CUDA;
     CUtensorMap mq, mk, mv;
@@ -472,9 +538,9 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
     pp.score_mode = scale > 0.f ? 0 : (scale < 0.f ? 1 : 2);
     pp.timeout_ns = g_timeout_ns.load();
     pp.test_flags = g_test_flags.load();
-    // persistent CTAs, one per SM (the kernel deals the units out itself)
-    const int64_t units = int64_t(pl.units_per_level) * pl.n_levels;
-    const int64_t grid = std::min<int64_t>(units, sm_count());
+    set_items(pp, pl, pb, ws);
+    // persistent CTAs, one per SM (the kernel deals the work items out itself)
+    const int64_t grid = std::min<int64_t>(prefill_items(pp), sm_count());
     return pb.window > 0 ? launch_prefill_kernel<T, DCH, true>(mq, mk, mv, pp, grid, stream)
                          : launch_prefill_kernel<T, DCH, false>(mq, mk, mv, pp, grid, stream);
 }
@@ -484,7 +550,7 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
 template <typename T, int DCH>
 attn_status_t launch_prefill_paged(const Problem& pb, const Plan& pl, const void* q, const void* kp,
                                    const void* vp, void* o, float* lse, float scale,
-                                   const PagedKV& pk, int64_t page_size, cudaStream_t stream) {
+                                   const PagedKV& pk, int64_t page_size, void* ws, cudaStream_t stream) {
     if (get_encoder() != ATTN_OK) return ATTN_ERR_CUDA;
     CUtensorMap mq, mk, mv;
     const uint32_t rows = uint32_t(std::min<int64_t>(page_size, 128));
@@ -511,17 +577,17 @@ attn_status_t launch_prefill_paged(const Problem& pb, const Plan& pl, const void
     pp.num_pages = pk.num_pages;
     pp.max_kv_len = pb.S;
     pp.page_shift = pk.page_shift;
-    const int64_t units = int64_t(pl.units_per_level) * pl.n_levels;
-    const int64_t grid = std::min<int64_t>(units, sm_count());
+    set_items(pp, pl, pb, ws);
+    const int64_t grid = std::min<int64_t>(prefill_items(pp), sm_count());
     return launch_prefill_kernel<T, DCH, false, true>(mq, mk, mv, pp, grid, stream);
 }
 
 template <typename T>
 attn_status_t run_prefill_tc(const Problem& pb, const Plan& pl, const void* q, const void* k,
-                             const void* v, void* o, float* lse, float scale,
+                             const void* v, void* o, float* lse, float scale, void* ws,
                              cudaStream_t stream) {
-    if (pl.dch == 1) return launch_prefill_tc<T, 1>(pb, pl, q, k, v, o, lse, scale, stream);
-    return launch_prefill_tc<T, 2>(pb, pl, q, k, v, o, lse, scale, stream);
+    if (pl.dch == 1) return launch_prefill_tc<T, 1>(pb, pl, q, k, v, o, lse, scale, ws, stream);
+    return launch_prefill_tc<T, 2>(pb, pl, q, k, v, o, lse, scale, ws, stream);
 }
 
 attn_status_t dispatch(const Problem& pb, const Plan& pl, const void* q, const void* k,
@@ -539,8 +605,8 @@ attn_status_t dispatch(const Problem& pb, const Plan& pl, const void* q, const v
         return run_decode<__half>(pb, pl, q, k, v, o, lse, scale, ws, stream);
     case ATTN_KERNEL_TCGEN05:
         if (pb.dt == ATTN_BF16)
-            return run_prefill_tc<__nv_bfloat16>(pb, pl, q, k, v, o, lse, scale, stream);
-        return run_prefill_tc<__half>(pb, pl, q, k, v, o, lse, scale, stream);
+            return run_prefill_tc<__nv_bfloat16>(pb, pl, q, k, v, o, lse, scale, ws, stream);
+        return run_prefill_tc<__half>(pb, pl, q, k, v, o, lse, scale, ws, stream);
     }
     return ATTN_ERR_INVALID_ARG;
 }
@@ -876,13 +942,13 @@ attn_status_t attn_cached_paged(const void* q, const void* k_pages, const void* 
         const bool bf16 = dtype == ATTN_BF16;
         if (pl.dch == 1)
             return bf16 ? launch_prefill_paged<__nv_bfloat16, 1>(pb, pl, q, k_pages, v_pages, o, lse, scale, pk,
-                                                                 page_size, s)
+                                                                 page_size, workspace, s)
                         : launch_prefill_paged<__half, 1>(pb, pl, q, k_pages, v_pages, o, lse, scale, pk,
-                                                          page_size, s);
+                                                          page_size, workspace, s);
         return bf16 ? launch_prefill_paged<__nv_bfloat16, 2>(pb, pl, q, k_pages, v_pages, o, lse, scale, pk,
-                                                             page_size, s)
+                                                             page_size, workspace, s)
                     : launch_prefill_paged<__half, 2>(pb, pl, q, k_pages, v_pages, o, lse, scale, pk,
-                                                      page_size, s);
+                                                      page_size, workspace, s);
     }
     if (dtype == ATTN_BF16)
         return run_decode<__nv_bfloat16>(pb, pl, q, k_pages, v_pages, o, lse, scale, workspace, s, &pk);
@@ -894,7 +960,7 @@ size_t attn_cached_paged_workspace_size(attn_dtype_t dtype, int64_t B, int64_t H
     if (Tnew < 0 || max_kv_len < Tnew) return 0;
     Plan pl;
     if (make_plan(paged_problem(dtype, B, H, Hkv, Tnew, d, max_kv_len), pl) != ATTN_OK) return 0;
-    return pl.kernel == ATTN_KERNEL_SPLITKV ? pl.ws_bytes : 0;
+    return pl.ws_bytes;
 }
 
 attn_status_t attn_prefill_local(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -1083,7 +1149,7 @@ extern "C" attn_status_t attn_cached_noalloc(const void* q, const void* k_hist,
     Problem pb{dtype, B, H, Hkv, Tnew, S, S_cap, d, start_pos, 1, true};
     if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
     Plan pl;
-    attn_status_t st = make_plan(pb, pl);
+    attn_status_t st = make_plan(pb, pl, ATTN_NOALLOC_SCRATCH_BYTES);
     if (st != ATTN_OK) return st;
     st = check_pointers(pb, q, k_hist, v_hist, o, lse);
     if (st != ATTN_OK) return st;

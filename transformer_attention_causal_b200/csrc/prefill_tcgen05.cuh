@@ -15,6 +15,10 @@
 // to persistent CTAs (one per SM) in a snake order; barrier phases keep
 // counting across a CTA's units, so the next unit's Q and first K/V copies
 // and its first Q.K^T overlap the current unit's last tiles and epilogue.
+// When the last pass would leave most CTAs idle, its units are cut into
+// `split` pieces along the key tiles (the split-KV idea of the decode kernel
+// applied to a prefill tail): each piece writes its O / l and log2-sum-exp
+// in fp32 to a workspace and prefill_merge_kernel combines them.
 //
 // Warp roles (12 warps):
 //   warp 0      TMA producer: per unit the Q tiles (once the previous unit's
@@ -39,6 +43,15 @@
 // TMEM) when the tile maximum exceeds it by more than 2^8 in the exp2 domain;
 // otherwise the stale maximum keeps every P below 256, exact after the final
 // division by l.
+//
+// The code of warpgroup 0 (producer, MMA issuer, paged-tail warp) holds no
+// 64-bit integer division or remainder by a run-time value.  Twice, such a
+// division added to that code (once executed per unit, once in a branch that
+// never ran for the failing calls) made the windowed MHA prefill wrong at d =
+// 128 with a window of about one key tile: the scores of a unit's second
+// slot, whose window starts one key tile after the first slot's, came out
+// wrong for that first tile, deterministically, while the same arithmetic in
+// 32-bit form gave correct results.  The mechanism was not found.
 #pragma once
 
 #include "ptx.cuh"
@@ -59,6 +72,12 @@ struct PrefillParams {
     int units_per_level;
     int n_levels;        // units = units_per_level * n_levels, heaviest level first
     int group;           // units of a level taken together (grouped_order)
+    // work items: units [0, n_whole) whole, then every later unit as `split`
+    // pieces over its key tiles (ws_o / ws_lse: a piece's fp32 O / l and
+    // m + log2 l per row, [piece][slot][128 rows][d] and [piece][slot][128])
+    int n_whole, split;
+    float* ws_o;
+    float* ws_lse;
     float scale_log2;    // |scale| * log2(e) (1 when scale = 0)
     int score_mode;      // 0: scale > 0; 1: scale < 0 (scores negated); 2: scale = 0 (scores zeroed)
     uint64_t timeout_ns;
@@ -285,6 +304,49 @@ __device__ __forceinline__ void prefill_unit(const PrefillParams& p, int unit, i
     slot[1] = prefill_slot<WINDOW>(p, h1, qb1, S, start);
 }
 
+// Work items: unit `item` while item < n_whole, then piece
+// (item - n_whole) % split of unit n_whole + (item - n_whole) / split.  A
+// piece keeps the key tiles [lo, hi) of its part of the unit's range; a slot
+// left with none is empty (n_kv = 0).  Returns the piece index, or -1 for a
+// whole unit.
+__host__ __device__ __forceinline__ int prefill_items(const PrefillParams& p) {
+    return p.n_whole + (p.units_per_level * p.n_levels - p.n_whole) * p.split;
+}
+
+template <bool WINDOW, bool PAGED>
+__device__ __forceinline__ int prefill_item(const PrefillParams& p, int item, int& b, int& kvh,
+                                            SlotInfo (&slot)[2]) {
+    if (item < p.n_whole) {
+        prefill_unit<WINDOW, PAGED>(p, item, b, kvh, slot);
+        return -1;
+    }
+    const int piece = item - p.n_whole;
+    const int part = piece % p.split;
+    prefill_unit<WINDOW, PAGED>(p, p.n_whole + piece / p.split, b, kvh, slot);
+    int n0 = 0x7fffffff, n1 = 0;
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+        if (slot[s].n_kv > 0) {
+            n0 = min(n0, slot[s].n_lo);
+            n1 = max(n1, slot[s].n_kv);
+        }
+    if (n1 == 0) return piece;
+    // 32-bit: a unit spans fewer than 2^26 key tiles (S * d * 2 < 2^40 with
+    // d >= 64, checked on the host), times part + 1 <= 4.  The warps of
+    // warpgroup 0 run no 64-bit division by a run-time value (see the note
+    // at the top of the kernel).
+    const int lo = n0 + (n1 - n0) * part / p.split;
+    const int hi = n0 + (n1 - n0) * (part + 1) / p.split;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        if (slot[s].n_kv == 0) continue;
+        slot[s].n_lo = max(slot[s].n_lo, lo);
+        slot[s].n_kv = min(slot[s].n_kv, hi);
+        if (slot[s].n_lo >= slot[s].n_kv) slot[s].n_lo = slot[s].n_kv = 0;
+    }
+    return piece;
+}
+
 // K or V tile n of sequence b, head kvh, from a paged pool: one TMA copy per
 // page the tile spans (min(P, 128) rows each).  Copies that start at or past
 // the sequence's end, and pages whose id is out of range (reported), are read
@@ -348,7 +410,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_units = p.units_per_level * p.n_levels;
+    const int n_items = prefill_items(p);
 
     // Persistent CTAs work through their units as one pipeline: every barrier
     // keeps counting phases across units (each role tracks its own counts),
@@ -394,10 +456,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 bool ok = true;
                 for (int pass = 0; ok; ++pass) {
                     const int unit = prefill_pass_unit(pass);
-                    if (unit >= n_units) break;
+                    if (unit >= n_items) break;
                     int b, kvh;
                     SlotInfo slot[2];
-                    prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                    prefill_item<WINDOW, PAGED>(p, unit, b, kvh, slot);
                     const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                     const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                      : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
@@ -460,10 +522,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 bool ok = true;
                 for (int pass = 0; ok; ++pass) {
                     const int unit = prefill_pass_unit(pass);
-                    if (unit >= n_units) break;
+                    if (unit >= n_items) break;
                     int b, kvh;
                     SlotInfo slot[2];
-                    prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                    prefill_item<WINDOW, PAGED>(p, unit, b, kvh, slot);
                     const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                     const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                      : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
@@ -473,6 +535,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                         ok = mbar_wait(smem_u32(&q_full[s]), qcount[s] & 1, p.timeout_ns, abort_flag);
                         ++qcount[s];
                     }
+                    if (nmax == 0) continue;   // a piece with no key tiles: nothing was loaded
                     if (ok) ok = mbar_wait(smem_u32(&kv_full[li % NST]), uint32_t((li / NST) & 1), p.timeout_ns,
                                            abort_flag);
                     if (!ok) break;
@@ -559,22 +622,22 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             // them, so with an even ring every use of a V stage is a V load
             // and kv_ready's phases follow kv_full's.
             static_assert(NST % 2 == 0, "V loads must keep to their own stages");
-            const int64_t copy_rows = min(int64_t(1) << p.page_shift, int64_t(128));
+            const int copy_shift = min(p.page_shift, 7);   // a copy brings min(P, 128) rows
             int64_t li = 0;
             bool ok = true;
             for (int pass = 0; ok; ++pass) {
                 const int unit = prefill_pass_unit(pass);
-                if (unit >= n_units) break;
+                if (unit >= n_items) break;
                 int b, kvh;
                 SlotInfo slot[2];
-                prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                prefill_item<WINDOW, PAGED>(p, unit, b, kvh, slot);
                 const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                 const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                  : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
                 const int n_loads = (p.test_flags & kTestSkipLoads) ? 0 : 2 * (nmax - nmin);
                 const int64_t L = slot[0].S;
                 // rows [L, end of the copy holding row L - 1) came from the pool
-                const int64_t tail_end = (L + copy_rows - 1) / copy_rows * copy_rows;
+                const int64_t tail_end = ((L + (int64_t(1) << copy_shift) - 1) >> copy_shift) << copy_shift;
                 for (int i = 0; i < n_loads && ok; ++i, ++li) {
                     if ((i & 1) == 0) continue;
                     const int st = int(li % NST);
@@ -615,14 +678,19 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
         bool ok = true;
         for (int pass = 0; ok; ++pass) {
             const int unit = prefill_pass_unit(pass);
-            if (unit >= n_units) break;
+            if (unit >= n_items) break;
             int b, kvh;
             SlotInfo slot[2];
-            prefill_unit<WINDOW, PAGED>(p, unit, b, kvh, slot);
+            const int piece = prefill_item<WINDOW, PAGED>(p, unit, b, kvh, slot);
             const SlotInfo sl = slot[s];
-            if (sl.n_kv == 0) continue;
+            if (sl.n_kv == 0) {
+                // a piece's slot with no key tiles: its partial weighs nothing
+                if (piece >= 0 && sl.q0 < p.Tq) p.ws_lse[(size_t(piece) * 2 + s) * 128 + row] = -INFINITY;
+                continue;
+            }
             const int64_t qpos = sl.start + sl.q0 + row;
             float m_run = -INFINITY, l = 0.f;
+            bool first = true;   // the slot's first key tile of this item
             for (int n = sl.n_lo; n < sl.n_kv; ++n) {
                 ok = mbar_wait(smem_u32(&s_full[s]), scount & 1, p.timeout_ns, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
@@ -636,7 +704,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tmem_ld32(tS + 32, r1);
                 tmem_ld32(tS + 64, r2);
                 tmem_ld32(tS + 96, r3);
-                tmem_wait_ld();
+                tmem_wait_ld(r0, r1, r2, r3);
                 if (p.score_mode != 0) {
                     // scale < 0 is attention on -S with |scale|; scale = 0 weighs
                     // every visible key alike (the mask below still applies)
@@ -670,7 +738,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
                 const float m_tile =
                     fmaxf(fmaxf(chunk_max(r0), chunk_max(r1)), fmaxf(chunk_max(r2), chunk_max(r3))) * c2;
-                if (n == sl.n_lo) {
+                if (first) {
+                    first = false;
                     m_run = m_tile;
                 } else {
                     const bool need = m_tile - m_run > kRescaleThreshold;
@@ -684,7 +753,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                         for (int cc = 0; cc < p.d; cc += 16) {
                             uint32_t x[16];
                             tmem_ld16(tO + cc, x);
-                            tmem_wait_ld();
+                            tmem_wait_ld(x);
 #pragma unroll
                             for (int e = 0; e < 16; ++e)
                                 x[e] = __float_as_uint(__uint_as_float(x[e]) * alpha);
@@ -697,8 +766,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 // before the last 64 are computed.  r* then hold P in fp32.
                 const float2 c2v = make_float2(c2, c2);
                 // a row that has seen no key yet (a window starting in a later
-                // tile) has m_run = -inf: its P must be 0, not NaN
-                const float m_use = WINDOW && m_run == -INFINITY ? 0.f : m_run;
+                // tile, or a piece's range ending before the row's first key)
+                // has m_run = -inf: its P must be 0, not NaN
+                const float m_use = m_run == -INFINITY ? 0.f : m_run;
                 const float2 negm = make_float2(-m_use, -m_use);
                 exp_chunk<T>(r0, c2v, negm, tS + 0);
                 exp_chunk<T>(r1, c2v, negm, tS + 16);
@@ -719,7 +789,29 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (ok) ok = mbar_wait(smem_u32(&o_done[s]), ocount & 1, p.timeout_ns, abort_flag);
             ++ocount;
             ok = __all_sync(0xffffffffu, ok);
-            if (ok) {
+            const int item = prefill_pass_unit(pass);
+            if (ok && item >= p.n_whole) {
+                // a piece: O / l and m + log2 l in fp32 for the merge (a row
+                // that saw no key of the piece has l = 0 and weighs nothing)
+                tc_fence_after();
+                const bool valid = sl.q0 + row < p.Tq;
+                const size_t prow = (size_t(item - p.n_whole) * 2 + s) * 128 + row;
+                float* wo = p.ws_o + prow * p.d;
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                for (int cc = 0; cc < p.d; cc += 16) {
+                    uint32_t x[16];
+                    tmem_ld16(tO + cc, x);
+                    tmem_wait_ld(x);
+                    if (valid) {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4)
+                            *reinterpret_cast<float4*>(wo + cc + e) =
+                                make_float4(__uint_as_float(x[e]) * inv, __uint_as_float(x[e + 1]) * inv,
+                                            __uint_as_float(x[e + 2]) * inv, __uint_as_float(x[e + 3]) * inv);
+                    }
+                }
+                if (valid) p.ws_lse[prow] = l > 0.f ? m_run + log2f(l) : -INFINITY;
+            } else if (ok) {
                 tc_fence_after();
                 const bool valid = sl.q0 + row < p.Tq;
                 const size_t orow = (size_t(b) * p.H + sl.h) * p.Tq + sl.q0 + row;
@@ -728,7 +820,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 for (int cc = 0; cc < p.d; cc += 16) {
                     uint32_t x[16];
                     tmem_ld16(tO + cc, x);
-                    tmem_wait_ld();
+                    tmem_wait_ld(x);
                     uint4 w0, w1;
                     w0.x = pack2<T>(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv);
                     w0.y = pack2<T>(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv);
@@ -754,6 +846,63 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// Merge of the pieces of the split units: per query row, the pieces' O_i and
+// m_i + log2 l_i (log2 domain) combine as O = sum_i 2^(lse_i - M) O_i / W with
+// M = max_i lse_i and W = sum_i 2^(lse_i - M); the row's log-sum-exp is
+// (M + log2 W) ln 2.  One warp per row, four d-columns per lane.  Launched as
+// a programmatic dependent of the prefill kernel: it waits for that grid's
+// results before reading them.
+constexpr int kMergeMaxSplit = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(128) prefill_merge_kernel(const PrefillParams p) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int n_tail = p.units_per_level * p.n_levels - p.n_whole;
+    const int64_t rid = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (rid >= int64_t(n_tail) * 256) return;
+    const int ui = int(rid >> 8), s = int(rid >> 7) & 1, r = int(rid & 127);
+    int b, kvh;
+    SlotInfo slot[2];
+    prefill_unit<false, false>(p, p.n_whole + ui, b, kvh, slot);
+    if (slot[s].q0 + r >= p.Tq) return;
+    float lse[kMergeMaxSplit];
+    float M = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMergeMaxSplit; ++i) {
+        lse[i] = i < p.split ? p.ws_lse[((size_t(ui) * p.split + i) * 2 + s) * 128 + r] : -INFINITY;
+        M = fmaxf(M, lse[i]);
+    }
+    float w[kMergeMaxSplit];
+    float W = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMergeMaxSplit; ++i) {
+        w[i] = lse[i] == -INFINITY ? 0.f : ex2(lse[i] - M);
+        W += w[i];
+    }
+    const float invW = W > 0.f ? 1.f / W : 0.f;
+    const size_t orow = (size_t(b) * p.H + slot[s].h) * p.Tq + slot[s].q0 + r;
+    const int c = lane * 4;
+    if (c < p.d) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kMergeMaxSplit; ++i) {
+            if (w[i] == 0.f) continue;
+            const float4 x = *reinterpret_cast<const float4*>(
+                p.ws_o + (((size_t(ui) * p.split + i) * 2 + s) * 128 + r) * p.d + c);
+            acc.x += w[i] * x.x;
+            acc.y += w[i] * x.y;
+            acc.z += w[i] * x.z;
+            acc.w += w[i] * x.w;
+        }
+        uint2 out;
+        out.x = pack2<T>(acc.x * invW, acc.y * invW);
+        out.y = pack2<T>(acc.z * invW, acc.w * invW);
+        *reinterpret_cast<uint2*>(static_cast<T*>(p.o) + orow * p.d + c) = out;
+    }
+    if (lane == 0 && p.lse) p.lse[orow] = W > 0.f ? (M + log2f(W)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace b200attn
