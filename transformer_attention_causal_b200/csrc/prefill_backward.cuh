@@ -184,7 +184,7 @@ __device__ __forceinline__ void bwd_store_row(uint32_t t_acc, int d, float mul, 
     for (int cc = first; cc < d; cc += step) {
         uint32_t x[16];
         tmem_ld16(t_acc + cc, x);
-        tmem_wait_ld(x);
+        tmem_wait_ld();
         uint4 w0, w1;
         w0.x = pack2<T>(__uint_as_float(x[0]) * mul, __uint_as_float(x[1]) * mul);
         w0.y = pack2<T>(__uint_as_float(x[2]) * mul, __uint_as_float(x[3]) * mul);
@@ -375,7 +375,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             uint32_t r[2][32];
             tmem_ld32(tS + 0, r[0]);
             tmem_ld32(tS + 32, r[1]);
-            tmem_wait_ld(r[0], r[1]);
+            tmem_wait_ld();
             // causal diagonal tile: query column i sees key row j only when i >= j;
             // with a window also only while i - j < w
             const int rel = row - (qt - kt) * 128 - 64 * half;   // column of i = j in this half
@@ -416,7 +416,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             for (int ch = 0; ch < 2; ++ch) {
                 uint32_t g[32];
                 tmem_ld32(tdP + 32 * ch, g);
-                tmem_wait_ld(g);
+                tmem_wait_ld();
                 float ddv[32];
                 lds32(dd + 128 * ch, ddv);
                 uint32_t pk[16];
@@ -703,7 +703,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             uint32_t r[2][32];
             tmem_ld32(tS + 0, r[0]);
             tmem_ld32(tS + 32, r[1]);
-            tmem_wait_ld(r[0], r[1]);
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(s_read));
@@ -742,7 +742,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             for (int ch = 0; ch < 2; ++ch) {
                 uint32_t g[32];
                 tmem_ld32(tdP + 32 * ch, g);
-                tmem_wait_ld(g);
+                tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float2 pp = make_float2(__uint_as_float(r[ch][2 * e]), __uint_as_float(r[ch][2 * e + 1]));

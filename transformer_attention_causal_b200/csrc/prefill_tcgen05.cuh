@@ -704,7 +704,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tmem_ld32(tS + 32, r1);
                 tmem_ld32(tS + 64, r2);
                 tmem_ld32(tS + 96, r3);
-                tmem_wait_ld(r0, r1, r2, r3);
+                tmem_wait_ld();
                 if (p.score_mode != 0) {
                     // scale < 0 is attention on -S with |scale|; scale = 0 weighs
                     // every visible key alike (the mask below still applies)
@@ -753,7 +753,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                         for (int cc = 0; cc < p.d; cc += 16) {
                             uint32_t x[16];
                             tmem_ld16(tO + cc, x);
-                            tmem_wait_ld(x);
+                            tmem_wait_ld();
 #pragma unroll
                             for (int e = 0; e < 16; ++e)
                                 x[e] = __float_as_uint(__uint_as_float(x[e]) * alpha);
@@ -801,7 +801,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 for (int cc = 0; cc < p.d; cc += 16) {
                     uint32_t x[16];
                     tmem_ld16(tO + cc, x);
-                    tmem_wait_ld(x);
+                    tmem_wait_ld();
                     if (valid) {
 #pragma unroll
                         for (int e = 0; e < 16; e += 4)
@@ -820,7 +820,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 for (int cc = 0; cc < p.d; cc += 16) {
                     uint32_t x[16];
                     tmem_ld16(tO + cc, x);
-                    tmem_wait_ld(x);
+                    tmem_wait_ld();
                     uint4 w0, w1;
                     w0.x = pack2<T>(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv);
                     w0.y = pack2<T>(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv);
