@@ -52,6 +52,8 @@ PREFILL = [
     (BF16, 1, 4, 4, 777, 80, 100, "tcgen05"),      # MHA row-tile pairs, d = 80
     (F16, 2, 2, 1, 1500, 64, 300, "tcgen05"),      # MQA, a window spanning several tiles
     (BF16, 1, 2, 2, 1024, 128, 128, "tcgen05"),    # window = one tile
+    (BF16, 1, 4, 4, 2048, 128, 120, "tcgen05"),    # MHA, each second slot's window starts a tile later
+    (BF16, 1, 2, 2, 1024, 128, 136, "tcgen05"),    # only rows 0-6 of a second slot see its first tile
     (BF16, 1, 2, 1, 600, 128, 1, "tcgen05"),       # only the own position
     (F32, 1, 4, 2, 300, 48, 17, "simt"),
     (BF16, 1, 2, 2, 200, 40, 50, "simt"),

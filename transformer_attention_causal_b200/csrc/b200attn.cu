@@ -473,12 +473,12 @@ attn_status_t run_decode(const Problem& pb, const Plan& pl, const void* q, const
     return ATTN_ERR_UNSUPPORTED;
 }
 
-template <typename T, int DCH, bool WINDOW, bool PAGED = false>
+template <typename T, int DCH, bool WINDOW, bool PAGED, bool SPLIT>
 attn_status_t launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk,
                                     const CUtensorMap& mv, const PrefillParams& pp, int64_t grid,
                                     cudaStream_t stream) {
     constexpr size_t smem = prefill_smem_bytes<DCH>();
-    constexpr auto kern = &prefill_tcgen05_kernel<T, DCH, WINDOW, PAGED>;
+    constexpr auto kern = &prefill_tcgen05_kernel<T, DCH, WINDOW, PAGED, SPLIT>;
     // the register split: warpgroup 0 at kPfRegsLow, the two softmax warpgroups at kPfRegsHigh
     if (const attn_status_t st =
             prepare_kernel<kern>(smem, kPfThreads, 128 * kPfRegsLow + 256 * kPfRegsHigh);
@@ -488,10 +488,12 @@ attn_status_t launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk
     if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
     if (pp.split <= 1) return ATTN_OK;
     // the pieces' merge, as a programmatic dependent (as the decode's combine)
+    // one warp per row: 256 rows per split unit
     const int64_t rows = int64_t(pp.units_per_level * pp.n_levels - pp.n_whole) * 256;
+    const int64_t warps_per_block = kMergeThreads / 32;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(unsigned((rows + 3) / 4));
-    cfg.blockDim = dim3(128);
+    cfg.gridDim = dim3(unsigned((rows + warps_per_block - 1) / warps_per_block));
+    cfg.blockDim = dim3(kMergeThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -541,8 +543,10 @@ attn_status_t launch_prefill_tc(const Problem& pb, const Plan& pl, const void* q
     set_items(pp, pl, pb, ws);
     // persistent CTAs, one per SM (the kernel deals the work items out itself)
     const int64_t grid = std::min<int64_t>(prefill_items(pp), sm_count());
-    return pb.window > 0 ? launch_prefill_kernel<T, DCH, true>(mq, mk, mv, pp, grid, stream)
-                         : launch_prefill_kernel<T, DCH, false>(mq, mk, mv, pp, grid, stream);
+    // pieces only in cached calls without a window (plan_tail_split)
+    if (pb.window > 0) return launch_prefill_kernel<T, DCH, true, false, false>(mq, mk, mv, pp, grid, stream);
+    return pp.split > 1 ? launch_prefill_kernel<T, DCH, false, false, true>(mq, mk, mv, pp, grid, stream)
+                        : launch_prefill_kernel<T, DCH, false, false, false>(mq, mk, mv, pp, grid, stream);
 }
 
 // The tensor-core prefill over a paged cache (chunked prefill): K/V maps over
@@ -579,7 +583,8 @@ attn_status_t launch_prefill_paged(const Problem& pb, const Plan& pl, const void
     pp.page_shift = pk.page_shift;
     set_items(pp, pl, pb, ws);
     const int64_t grid = std::min<int64_t>(prefill_items(pp), sm_count());
-    return launch_prefill_kernel<T, DCH, false, true>(mq, mk, mv, pp, grid, stream);
+    return pp.split > 1 ? launch_prefill_kernel<T, DCH, false, true, true>(mq, mk, mv, pp, grid, stream)
+                        : launch_prefill_kernel<T, DCH, false, true, false>(mq, mk, mv, pp, grid, stream);
 }
 
 template <typename T>

@@ -313,10 +313,10 @@ __host__ __device__ __forceinline__ int prefill_items(const PrefillParams& p) {
     return p.n_whole + (p.units_per_level * p.n_levels - p.n_whole) * p.split;
 }
 
-template <bool WINDOW, bool PAGED>
+template <bool WINDOW, bool PAGED, bool SPLIT>
 __device__ __forceinline__ int prefill_item(const PrefillParams& p, int item, int& b, int& kvh,
                                             SlotInfo (&slot)[2]) {
-    if (item < p.n_whole) {
+    if (!SPLIT || item < p.n_whole) {
         prefill_unit<WINDOW, PAGED>(p, item, b, kvh, slot);
         return -1;
     }
@@ -383,7 +383,9 @@ __device__ __forceinline__ int prefill_pass_unit(int k) {
                         : (k + 1) * int(gridDim.x) - 1 - int(blockIdx.x);
 }
 
-template <typename T, int DCH, bool WINDOW, bool PAGED>
+// SPLIT: the launch has pieces (n_whole < units); the kernels of launches
+// without them carry no piece code (it cost the BitNet-3B prefill 4 %).
+template <typename T, int DCH, bool WINDOW, bool PAGED, bool SPLIT>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -459,7 +461,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     if (unit >= n_items) break;
                     int b, kvh;
                     SlotInfo slot[2];
-                    prefill_item<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                    prefill_item<WINDOW, PAGED, SPLIT>(p, unit, b, kvh, slot);
                     const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                     const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                      : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
@@ -525,7 +527,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                     if (unit >= n_items) break;
                     int b, kvh;
                     SlotInfo slot[2];
-                    prefill_item<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                    prefill_item<WINDOW, PAGED, SPLIT>(p, unit, b, kvh, slot);
                     const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                     const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                      : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
@@ -630,7 +632,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (unit >= n_items) break;
                 int b, kvh;
                 SlotInfo slot[2];
-                prefill_item<WINDOW, PAGED>(p, unit, b, kvh, slot);
+                prefill_item<WINDOW, PAGED, SPLIT>(p, unit, b, kvh, slot);
                 const int nmax = max(slot[0].n_kv, slot[1].n_kv);
                 const int nmin = slot[0].n_kv == 0 ? slot[1].n_lo
                                  : slot[1].n_kv == 0 ? slot[0].n_lo : min(slot[0].n_lo, slot[1].n_lo);
@@ -681,11 +683,11 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (unit >= n_items) break;
             int b, kvh;
             SlotInfo slot[2];
-            const int piece = prefill_item<WINDOW, PAGED>(p, unit, b, kvh, slot);
+            const int piece = prefill_item<WINDOW, PAGED, SPLIT>(p, unit, b, kvh, slot);
             const SlotInfo sl = slot[s];
             if (sl.n_kv == 0) {
                 // a piece's slot with no key tiles: its partial weighs nothing
-                if (piece >= 0 && sl.q0 < p.Tq) p.ws_lse[(size_t(piece) * 2 + s) * 128 + row] = -INFINITY;
+                if (SPLIT && piece >= 0 && sl.q0 < p.Tq) p.ws_lse[(size_t(piece) * 2 + s) * 128 + row] = -INFINITY;
                 continue;
             }
             const int64_t qpos = sl.start + sl.q0 + row;
@@ -790,7 +792,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
             ++ocount;
             ok = __all_sync(0xffffffffu, ok);
             const int item = prefill_pass_unit(pass);
-            if (ok && item >= p.n_whole) {
+            if (SPLIT && ok && item >= p.n_whole) {
                 // a piece: O / l and m + log2 l in fp32 for the merge (a row
                 // that saw no key of the piece has l = 0 and weighs nothing)
                 tc_fence_after();
@@ -851,52 +853,59 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
 // Merge of the pieces of the split units: per query row, the pieces' O_i and
 // m_i + log2 l_i (log2 domain) combine as O = sum_i 2^(lse_i - M) O_i / W with
 // M = max_i lse_i and W = sum_i 2^(lse_i - M); the row's log-sum-exp is
-// (M + log2 W) ln 2.  One warp per row, four d-columns per lane.  Launched as
-// a programmatic dependent of the prefill kernel: it waits for that grid's
+// (M + log2 W) ln 2.  One warp per row, four d-columns per lane, four rows
+// per block.  (Measured against fewer, longer-lived warps that walk several
+// rows each, or decode their unit once for 16 rows: both slower.)  Launched
+// as a programmatic dependent of the prefill kernel: it waits for that grid's
 // results before reading them.
 constexpr int kMergeMaxSplit = 4;
+constexpr int kMergeThreads = 128;
 
 template <typename T>
-__global__ void __launch_bounds__(128) prefill_merge_kernel(const PrefillParams p) {
+__global__ void __launch_bounds__(kMergeThreads) prefill_merge_kernel(const PrefillParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int n_tail = p.units_per_level * p.n_levels - p.n_whole;
-    const int64_t rid = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
+    const int64_t rid = int64_t(blockIdx.x) * (kMergeThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (rid >= int64_t(n_tail) * 256) return;
     const int ui = int(rid >> 8), s = int(rid >> 7) & 1, r = int(rid & 127);
     int b, kvh;
     SlotInfo slot[2];
     prefill_unit<false, false>(p, p.n_whole + ui, b, kvh, slot);
-    if (slot[s].q0 + r >= p.Tq) return;
+    const int h = s ? slot[1].h : slot[0].h, q0 = s ? slot[1].q0 : slot[0].q0;   // no indexed local array
+    if (q0 + r >= p.Tq) return;
+    // every piece's row is loaded at once (one memory round trip, not one for
+    // the weights and another for the rows); a piece whose slot had no key
+    // tile left its row unwritten, so its weight selects it away rather than
+    // multiplying whatever the row holds
+    const int c = lane * 4;
     float lse[kMergeMaxSplit];
+    float4 x[kMergeMaxSplit];
+#pragma unroll
+    for (int i = 0; i < kMergeMaxSplit; ++i) {
+        const size_t prow = ((size_t(ui) * p.split + i) * 2 + s) * 128 + r;
+        lse[i] = i < p.split ? p.ws_lse[prow] : -INFINITY;
+        x[i] = i < p.split && c < p.d ? *reinterpret_cast<const float4*>(p.ws_o + prow * p.d + c)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float M = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < kMergeMaxSplit; ++i) {
-        lse[i] = i < p.split ? p.ws_lse[((size_t(ui) * p.split + i) * 2 + s) * 128 + r] : -INFINITY;
-        M = fmaxf(M, lse[i]);
-    }
-    float w[kMergeMaxSplit];
+    for (int i = 0; i < kMergeMaxSplit; ++i) M = fmaxf(M, lse[i]);
     float W = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < kMergeMaxSplit; ++i) {
-        w[i] = lse[i] == -INFINITY ? 0.f : ex2(lse[i] - M);
-        W += w[i];
+        const bool live = lse[i] != -INFINITY;
+        const float w = live ? ex2(lse[i] - M) : 0.f;
+        W += w;
+        acc.x += live ? w * x[i].x : 0.f;
+        acc.y += live ? w * x[i].y : 0.f;
+        acc.z += live ? w * x[i].z : 0.f;
+        acc.w += live ? w * x[i].w : 0.f;
     }
     const float invW = W > 0.f ? 1.f / W : 0.f;
-    const size_t orow = (size_t(b) * p.H + slot[s].h) * p.Tq + slot[s].q0 + r;
-    const int c = lane * 4;
+    const size_t orow = (size_t(b) * p.H + h) * p.Tq + q0 + r;
     if (c < p.d) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < kMergeMaxSplit; ++i) {
-            if (w[i] == 0.f) continue;
-            const float4 x = *reinterpret_cast<const float4*>(
-                p.ws_o + (((size_t(ui) * p.split + i) * 2 + s) * 128 + r) * p.d + c);
-            acc.x += w[i] * x.x;
-            acc.y += w[i] * x.y;
-            acc.z += w[i] * x.z;
-            acc.w += w[i] * x.w;
-        }
         uint2 out;
         out.x = pack2<T>(acc.x * invW, acc.y * invW);
         out.y = pack2<T>(acc.z * invW, acc.w * invW);
