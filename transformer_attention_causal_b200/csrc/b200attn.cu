@@ -157,9 +157,9 @@ int64_t first_tile_keys(const Problem& pb) {
 // them when U < g).  When R is at most half the CTAs, those units are cut into
 // `split` pieces of at least 4 key tiles each (at most kMergeMaxSplit,
 // R * split <= g), so the last pass costs about 1 / split of a unit instead of
-// a whole one while the other CTAs would idle.  Only calls of at most 8 full passes, where that tail is worth the
-// pieces' fp32 partials and the merge launch.  The pieces' workspace must fit
-// `ws_cap` (fewer pieces otherwise).
+// a whole one while the other CTAs would idle.  Only calls of at most 8 full
+// passes, where that tail is worth the pieces' fp32 partials and the merge
+// launch.  The pieces' workspace must fit `ws_cap` (fewer pieces otherwise).
 void plan_tail_split(const Problem& pb, Plan& pl, size_t ws_cap) {
     pl.n_whole = pl.units_per_level * pl.n_levels;
     pl.split = 1;
@@ -487,8 +487,8 @@ attn_status_t launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk
     kern<<<unsigned(grid), kPfThreads, smem, stream>>>(mq, mk, mv, pp);
     if (launch_status() != ATTN_OK) return ATTN_ERR_CUDA;
     if (pp.split <= 1) return ATTN_OK;
-    // the pieces' merge, as a programmatic dependent (as the decode's combine)
-    // one warp per row: 256 rows per split unit
+    // the pieces' merge, as a programmatic dependent (as the decode's
+    // combine): one warp per row, 256 rows per split unit
     const int64_t rows = int64_t(pp.units_per_level * pp.n_levels - pp.n_whole) * 256;
     const int64_t warps_per_block = kMergeThreads / 32;
     cudaLaunchConfig_t cfg{};
