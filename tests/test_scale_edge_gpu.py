@@ -75,6 +75,7 @@ CACHED = [
     # dtype, B, H, Hkv, Tnew, start_pos, S, d, kernel
     (BF16, 2, 8, 2, 1, 999, 1000, 128, "splitkv"),
     (F16, 2, 8, 1, 200, 300, 500, 128, "tcgen05"),
+    (BF16, 1, 8, 2, 130, 1000, 1130, 64, "tcgen05"),   # 8 units, each cut into 2 pieces of its keys
 ]
 
 
