@@ -88,7 +88,9 @@ typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1, ATTN_F16 = 2 } attn_dtype_t;
 typedef enum {
     ATTN_KERNEL_NONE = 0,        /* empty problem: nothing launched            */
     ATTN_KERNEL_SIMT = 1,        /* float32 CUDA-core kernel (any d <= 256)    */
-    ATTN_KERNEL_TCGEN05 = 2,     /* TMA + tcgen05/TMEM fused prefill kernel    */
+    ATTN_KERNEL_TCGEN05 = 2,     /* TMA + tcgen05/TMEM fused prefill kernel    *
+                                  * (+ the merge of a cached call's key-range  *
+                                  * pieces, when its last pass is cut)         */
     ATTN_KERNEL_SPLITKV = 3      /* split-KV decode kernel + LSE combine       */
 } attn_kernel_t;
 
