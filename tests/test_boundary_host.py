@@ -116,6 +116,26 @@ def test_cached_reports_a_short_workspace(lib):
     assert cached(lib, ws=MISALIGNED, ws_bytes=need, **args) == INVALID
 
 
+def test_chunked_prefill_pieces_need_their_workspace(lib):
+    """A chunked prefill whose last pass is cut into pieces needs the
+    workspace attn_cached_workspace_size reports; less is rejected before
+    anything is launched (host only: the pointers are never dereferenced)."""
+    F16 = 2
+    args = dict(dt=F16, B=32, H=8, Hkv=1, Tnew=512, S=4096, S_cap=4096, d=128, start_pos=3584)
+    need = lib.attn_cached_workspace_size(F16, 32, 8, 1, 512, 4096, 128, 3584)
+    assert need > 0
+    assert cached(lib, ws=None, ws_bytes=0, **args) == WORKSPACE
+    assert cached(lib, ws=FAKE, ws_bytes=need - 1, **args) == WORKSPACE
+    assert cached(lib, ws=MISALIGNED, ws_bytes=need, **args) == INVALID
+    # the paged form, planned at its length bound
+    need_p = lib.attn_cached_paged_workspace_size(F16, 32, 8, 1, 512, 128, 4096)
+    assert need_p == need
+    pargs = dict(dt=F16, B=32, H=8, Hkv=1, Tnew=512, d=128, max_pages=32, num_pages=1024,
+                 page_size=128, max_kv_len=4096)
+    assert paged(lib, ws=None, ws_bytes=0, **pargs) == WORKSPACE
+    assert paged(lib, ws=FAKE, ws_bytes=need_p - 1, **pargs) == WORKSPACE
+
+
 def test_empty_problems_are_a_no_op(lib):
     # B * H * Tq == 0: nothing is launched, null pointers allowed
     assert prefill(lib, q=None, k=None, v=None, o=None, B=0) == 0
